@@ -1,0 +1,595 @@
+#!/usr/bin/env python
+"""Benchmark of the QSA layer (libqsa) on B200.
+
+One step = one pass of the whole layer over one batch of seeded synthetic input:
+  prefill (headline, 1,048,576-token context, last 16,384-token chunk, batch 1):
+      compress the chunk's indexer keys -> score + select (top-512 + tail) -> sparse attention
+  decode (reported beside it, 1,048,576-token context, 4 sequences x 4 positions):
+      compress the new block -> score + select -> split-K sparse attention -> combine
+The settings are those of the article "Qwen's million-token window has a 2,048-token keyhole",
+section "Three speed claims, three different experiments".  The dense paged-GQA kernel of the
+same library runs on the same pools for the sparse/dense ratio, and the fp64 oracle is timed on
+the host cores as a baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs an independent replica of the
+workload (the layer shards by sequence with no data-path collective); the timed region is
+bracketed by a barrier and synchronisation and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QSA prefill tok/s and decode µs/step at 1M ctx; % of HBM/tensor roofline"
+PREFILL = "C4"
+DECODE = "C5"
+
+
+# ------------------------------------------------------------------------------------ helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), tf=float(d["bf16_tflops"]),
+                    tf_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, tf=1590.0, tf_sus=1400.0, src="fallback")
+
+
+def positions_of(t: int, topk: int = 512) -> int:
+    """Token positions attended by query position t: selected blocks plus the clipped tail."""
+    n = min(topk, t // 4)
+    return 4 * n + (t % 4) + 1
+
+
+def algorithmic(c, q_pos):
+    """Useful work per step (bytes or flops) of each stage, as defined for the roofline."""
+    import numpy as np
+
+    t = np.asarray(q_pos, dtype=np.int64)
+    kv_row = c.Hkv * c.D * 2  # bytes of one K (or V) position row, all kv heads
+    pos = np.array([positions_of(int(x), c.topk) for x in t], dtype=np.int64)
+    per_seq_max = t.reshape(c.batch, -1).max(axis=1)
+    return {
+        "compress_bytes": c.num_q * c.Di * 2 + (c.num_q // 4) * c.Di * 2,
+        "score_flops": int(2 * c.Hi * c.Di * (t // 4).sum()),
+        "score_bytes_decode": int(((per_seq_max // 4) * c.Di * 2).sum()),
+        "attn_bytes": int(pos.sum() * kv_row * 2),
+        "attn_flops": int(pos.sum() * 4 * c.Hq * c.D),
+        "dense_flops": int((4 * c.Hq * c.D * (t + 1)).sum()),
+        "dense_bytes_decode": int(((per_seq_max + 1) * kv_row * 2).sum()),
+    }
+
+
+class Clocks:
+    """nvidia-smi samples (200 ms) during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="qsa_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}", "--format=csv,noheader",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if not self.path or not os.path.exists(self.path):
+            return out
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1].split()[0]))
+                smax.append(float(f[2].split()[0]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if sm:
+            out.update(sm_mhz=statistics.median(sm), sm_max_mhz=max(smax), samples=len(sm))
+        out["reasons"] = sorted(reasons)
+        return out
+
+
+def traffic_for(kernel_file: str, key: str):
+    """dram bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(key)
+    except (OSError, ValueError):
+        return None
+    if not d:
+        return None
+    src = os.path.join(ROOT, "learned_block_sparse_qsa_b200", "csrc", kernel_file)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return d["bytes_per_launch"] if d.get("source_sha") == h else None
+
+
+# ------------------------------------------------------------------------------------ workload
+
+class Workload:
+    """Device inputs + runner for one config (the prefix of the context already compressed)."""
+
+    def __init__(self, name: str, device):
+        import torch
+
+        from learned_block_sparse_qsa_b200 import QsaConfig, QsaRunner
+        from qsa_synth import CONFIGS
+        from qsa_synth.device import DeviceInputs
+
+        self.torch = torch
+        self.c = c = CONFIGS[name]
+        self.di = d = DeviceInputs(c, integer=False, device=device)
+        self.cfg = QsaConfig.make(c.Hq, c.Hkv, c.D, c.Di, topk=c.topk)
+        self.runner = QsaRunner(self.cfg, device)
+        self.b = self.runner.batch(batch=c.batch, num_q=c.num_q, max_pages=c.max_pages,
+                                   num_pages=c.num_pages, max_pos=c.ctx - 1, q_seq=d.q_seq,
+                                   q_pos=d.q_pos, page_table=d.page_table)
+        self.sel = torch.empty(c.num_q, c.topk + 1, dtype=torch.int32, device=device)
+        self.n_sel = torch.empty(c.num_q, dtype=torch.int32, device=device)
+        self.out = torch.empty_like(d.q)
+        for s in range(c.batch):
+            rows, seq, pos = d.prefix_rows(s)
+            if rows.shape[0]:
+                self.runner.compress(self.b, rows, seq, pos, d.kcomp_pool)
+        torch.cuda.synchronize()
+        self.q_pos_host = d.host.rows()[1]
+
+    def stage_calls(self, decode: bool):
+        """The step as a list of (stage name, callable) on the current stream."""
+        from learned_block_sparse_qsa_b200 import (QSA_OP_SPARSE_ATTN_DECODE, qsa_sparse_attn_decode,
+                                                   qsa_sparse_attn_prefill)
+
+        d, r, b, cfg = self.di, self.runner, self.b, self.cfg
+        calls = [("compress", lambda: r.compress(b, d.idx_k_new, d.new_seq, d.new_pos, d.kcomp_pool)),
+                 ("score_topk", lambda: r.select(b, d.idx_q, d.idx_w, d.kcomp_pool, self.sel, self.n_sel))]
+        if decode:
+            ws, n = r.workspace(b, QSA_OP_SPARSE_ATTN_DECODE, 0)
+            calls.append(("sparse_attn", lambda: qsa_sparse_attn_decode(
+                cfg, b, d.q, d.k_pool, d.v_pool, self.sel, self.n_sel, self.out, None, 0, ws, n)))
+        else:
+            calls.append(("sparse_attn", lambda: qsa_sparse_attn_prefill(
+                cfg, b, d.q, d.k_pool, d.v_pool, self.sel, self.n_sel, self.out)))
+        return calls
+
+    def step(self, decode: bool):
+        for _, f in self.stage_calls(decode):
+            f()
+
+
+def time_steps(w: Workload, decode: bool, steps: int, warmup: int, dist, flush=None):
+    """Per-stage and whole-step device times (ms) over `steps` timed steps."""
+    torch = w.torch
+    calls = w.stage_calls(decode)
+    for _ in range(warmup):
+        for _, f in calls:
+            f()
+    torch.cuda.synchronize()
+    names = [n for n, _ in calls]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        ev[i][0].record()
+        for j, (_, f) in enumerate(calls):
+            f()
+            ev[i][j + 1].record()
+    t1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    stage_ms = {n: 0.0 for n in names}
+    step_ms = []
+    for i in range(steps):
+        for j, n in enumerate(names):
+            stage_ms[n] += ev[i][j].elapsed_time(ev[i][j + 1])
+        step_ms.append(ev[i][0].elapsed_time(ev[i][-1]))
+    return {n: v / steps for n, v in stage_ms.items()}, step_ms, t0.elapsed_time(t1)
+
+
+def max_over_ranks(x: float, dist) -> float:
+    if not dist:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def graph_decode_us(w: Workload, steps: int, warmup: int, flush):
+    """Decode step captured in one CUDA graph; mean replay time (us), L2 flushed in between."""
+    torch = w.torch
+    for _ in range(max(warmup, 1)):
+        w.step(True)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        w.step(True)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        w.step(True)
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    us = [a.elapsed_time(b) * 1000 for a, b in ts]
+    del g
+    return statistics.mean(us), us
+
+
+def e2e_prefill(w: Workload, steps: int, warmup: int):
+    """Whole step through the public API with host inputs: H2D of the chunk's inputs (queries,
+    indexer queries/weights/keys, the new K/V pages), the layer, D2H of the output."""
+    torch = w.torch
+    c, d = w.c, w.di
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    hq, hiq, hiw, hik = pin(d.q), pin(d.idx_q), pin(d.idx_w), pin(d.idx_k_new)
+    lp0, lp1 = c.ctx_start // 64, (c.ctx - 1) // 64 + 1
+    pages = d.page_table[0, lp0:lp1].long()
+    hk, hv = pin(d.k_pool[pages]), pin(d.v_pool[pages])
+    pages_h = pages.cpu().tolist()
+    hout = torch.empty(d.q.shape, dtype=d.q.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hiq, hiw, hik, hk, hv))
+    d2h = hout.numel() * hout.element_size()
+
+    def one():
+        d.q.copy_(hq, non_blocking=True)
+        d.idx_q.copy_(hiq, non_blocking=True)
+        d.idx_w.copy_(hiw, non_blocking=True)
+        d.idx_k_new.copy_(hik, non_blocking=True)
+        for i, p in enumerate(pages_h):
+            d.k_pool[p].copy_(hk[i], non_blocking=True)
+            d.v_pool[p].copy_(hv[i], non_blocking=True)
+        w.step(False)
+        hout.copy_(w.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return ms, h2d, d2h
+
+
+def e2e_decode(w: Workload, steps: int, warmup: int):
+    torch = w.torch
+    c, d = w.c, w.di
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    hq, hiq, hiw, hik = pin(d.q), pin(d.idx_q), pin(d.idx_w), pin(d.idx_k_new)
+    q_pos = d.q_pos.cpu().long()
+    q_seq = d.q_seq.cpu().long()
+    pages = d.page_table.cpu()[q_seq, q_pos // 64].long()
+    slots = (q_pos % 64).long()
+    hk = pin(d.k_pool[pages.cuda(), slots.cuda()])
+    hv = pin(d.v_pool[pages.cuda(), slots.cuda()])
+    kv_dst = list(zip(pages.tolist(), slots.tolist()))
+    hout = torch.empty(d.q.shape, dtype=d.q.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hiq, hiw, hik, hk, hv))
+    d2h = hout.numel() * hout.element_size()
+
+    def one():
+        d.q.copy_(hq, non_blocking=True)
+        d.idx_q.copy_(hiq, non_blocking=True)
+        d.idx_w.copy_(hiw, non_blocking=True)
+        d.idx_k_new.copy_(hik, non_blocking=True)
+        for i, (p, s) in enumerate(kv_dst):
+            d.k_pool[p, s].copy_(hk[i], non_blocking=True)
+            d.v_pool[p, s].copy_(hv[i], non_blocking=True)
+        w.step(True)
+        hout.copy_(w.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) * 1000 / steps, h2d, d2h
+
+
+def dense_time_ms(w: Workload, decode: bool, reps: int, flush=None):
+    torch = w.torch
+    d = w.di
+    out = torch.empty_like(w.out)
+    w.runner.dense(w.b, q=d.q, k_pool=d.k_pool, v_pool=d.v_pool, out=out, decode=decode)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        if flush:
+            flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        w.runner.dense(w.b, q=d.q, k_pool=d.k_pool, v_pool=d.v_pool, out=out, decode=decode)
+        b.record()
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in ts)
+
+
+# ------------------------------------------------------------------------------------ oracle
+
+def oracle_prefill_baseline(rows_per_step: int, steps: int):
+    """The fp64 oracle on the host cores, on a bounded sample of the prefill workload: the
+    chunk's compression once, then selection + attention for evenly spaced query rows."""
+    import numpy as np
+
+    from oracle import qsa_oracle as orc
+    from qsa_synth import CONFIGS, HostInputs
+
+    c = CONFIGS[PREFILL]
+    h = HostInputs(c)
+    kc_prefix = orc.compress(h.idx_k(0, 0, c.ctx_start))       # setup, not timed
+    chunk_keys = h.idx_k(0, c.ctx_start, c.ctx)
+    t0 = time.perf_counter()
+    kc_chunk = orc.compress(chunk_keys)
+    t_compress = time.perf_counter() - t0
+    kc = np.concatenate([kc_prefix, kc_chunk])
+    n = rows_per_step * steps
+    rows = np.linspace(0, c.num_q - 1, n).round().astype(int)
+    _, q_pos = h.rows()
+    iq, iw, qq = h.idx_q(rows), h.idx_w(rows), h.q(rows)
+    t_rows = 0.0
+    per_step = []
+    for i, r in enumerate(rows):
+        t = int(q_pos[r])
+        a = time.perf_counter()
+        sel, _ = orc.qsa_select(kc, iq[i], iw[i], t)
+        pos = orc.expand(sel, t)
+        b = time.perf_counter()
+        k, v = h.kv(0, pos)                                      # input regeneration, not timed
+        c0 = time.perf_counter()
+        orc.attend(qq[i], k, v)
+        e = time.perf_counter()
+        t_rows += (b - a) + (e - c0)
+        per_step.append((b - a) + (e - c0))
+    per_token = t_compress / c.num_q + t_rows / n
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count() or 1
+    return dict(value=1.0 / per_token, unit="tok/s", cores=int(cores), kind="oracle",
+                sample=f"{n} evenly spaced query rows of the {c.num_q}-token chunk at "
+                       f"{c.ctx}-token context (selection + attention each) plus the chunk's "
+                       f"compression; tok/s extrapolated from seconds per token",
+                seconds=t_compress + t_rows)
+
+
+# ------------------------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    peaks = load_peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps = max(1, args.steps)
+        base = oracle_prefill_baseline(rows_per_step=4, steps=steps)
+        from qsa_synth import CONFIGS
+
+        c = CONFIGS[PREFILL]
+        line = {"metric": METRIC, "value": base["value"], "unit": "tok/s", "impl": "reference",
+                "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+                "ms_per_step": 1000.0 * base["seconds"] / steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": c.name, "batch": c.batch, "ctx": c.ctx, "chunk": c.n_new},
+                "cpu_baseline": {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": base["value"], "unit": "tok/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_index = int(vis.split(",")[local]) if vis and vis.split(",")[local].isdigit() else local
+    l2_flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = lambda: l2_flush_buf.zero_()  # noqa: E731
+
+    # ---------------------------------------------------------------- prefill (headline)
+    w = Workload(PREFILL, dev)
+    c = w.c
+    work = algorithmic(c, w.q_pos_host)
+    with Clocks(gpu_index) as clk:
+        stage_ms, step_ms, total_ms = time_steps(w, False, args.steps, args.warmup, dist)
+    clocks = clk.summary()
+    total_ms = max_over_ranks(total_ms, dist)
+    ms_step = total_ms / args.steps
+    value = world * c.num_q * args.steps / (total_ms / 1000.0)
+    launches_per_step = 3
+    stages = {
+        "compress": dict(ms=stage_ms["compress"], bound="hbm", unit="GB/s",
+                         achieved=work["compress_bytes"] / (stage_ms["compress"] * 1e-3) / 1e9,
+                         peak=peaks["hbm"], kernel_file="compress.cu"),
+        "score_topk": dict(ms=stage_ms["score_topk"], bound="tensor", unit="TFLOP/s",
+                           achieved=work["score_flops"] / (stage_ms["score_topk"] * 1e-3) / 1e12,
+                           peak=peaks["tf_sus"], kernel_file="score.cu"),
+        "sparse_attn": dict(ms=stage_ms["sparse_attn"], bound="hbm", unit="GB/s",
+                            achieved=work["attn_bytes"] / (stage_ms["sparse_attn"] * 1e-3) / 1e9,
+                            peak=peaks["hbm"], kernel_file="attn.cu"),
+    }
+    for s in stages.values():
+        s["frac"] = s["achieved"] / s["peak"]
+    dom = max(stages, key=lambda k: stages[k]["ms"])
+    ds = stages[dom]
+    per_launch = {"compress": work["compress_bytes"], "score_topk": work["score_flops"],
+                  "sparse_attn": work["attn_bytes"]}[dom]
+    roofline = {"bound": ds["bound"], "achieved": ds["achieved"], "peak": ds["peak"], "unit": ds["unit"],
+                "frac": ds["frac"], "kernel": dom, "work_per_launch": per_launch,
+                "peak_source": peaks["src"] + (" sustained" if ds["bound"] == "tensor" else ""),
+                "traffic": traffic_for(ds["kernel_file"], f"{dom}@{PREFILL}")}
+    path_roof_ms = (work["compress_bytes"] / (peaks["hbm"] * 1e9) + work["score_flops"] / (peaks["tf_sus"] * 1e12)
+                    + work["attn_bytes"] / (peaks["hbm"] * 1e9)) * 1e3
+    e2e_ms, h2d, d2h = e2e_prefill(w, max(3, args.steps // 3), 2)
+    dense_ms = dense_time_ms(w, False, 1)
+    del w
+    torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- decode
+    wd = Workload(DECODE, dev)
+    cd = wd.c
+    workd = algorithmic(cd, wd.q_pos_host)
+    dsteps = max(50, 5 * args.steps)
+    dstage_ms, dstep_ms, _ = time_steps(wd, True, dsteps, args.warmup, dist, flush=flush)
+    graph_us, _ = graph_decode_us(wd, dsteps, args.warmup, flush)
+    graph_us = max_over_ranks(graph_us, dist)
+    d_e2e_us, dh2d, dd2h = e2e_decode(wd, dsteps, args.warmup)
+    dense_dec_ms = dense_time_ms(wd, True, 5, flush)
+    dstages = {
+        "score_topk": dict(ms=dstage_ms["score_topk"], bound="hbm", unit="GB/s",
+                           achieved=workd["score_bytes_decode"] / (dstage_ms["score_topk"] * 1e-3) / 1e9,
+                           peak=peaks["hbm"]),
+        "sparse_attn": dict(ms=dstage_ms["sparse_attn"], bound="hbm", unit="GB/s",
+                            achieved=workd["attn_bytes"] / (dstage_ms["sparse_attn"] * 1e-3) / 1e9,
+                            peak=peaks["hbm"]),
+        "compress": dict(ms=dstage_ms["compress"]),
+    }
+    for s in dstages.values():
+        if "achieved" in s:
+            s["frac"] = s["achieved"] / s["peak"]
+    dpath_roof_us = (workd["score_bytes_decode"] + workd["attn_bytes"]) / (peaks["hbm"] * 1e9) * 1e6
+    del wd
+    torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1:
+        base = oracle_prefill_baseline(rows_per_step=8, steps=4)
+        cpu = {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded counter-based N(0,1) stand-in + 64 planted needle blocks",
+            "config": {"workload": c.name, "batch": c.batch, "ctx": c.ctx, "chunk": c.n_new,
+                       "q_heads": c.Hq, "kv_heads": c.Hkv, "head_dim": c.D, "idx_heads": c.Hi,
+                       "idx_dim": c.Di, "topk_blocks": c.topk, "page_tokens": c.page,
+                       "l2": "inputs larger than L2 (2 GiB paged KV gathered per step); decode "
+                             "steps flush L2 (256 MiB write) between timed steps",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roofline,
+            "stages_ms": {k: v["ms"] for k, v in stages.items()},
+            "stages": {k: {kk: vv for kk, vv in v.items() if kk != "kernel_file"} for k, v in stages.items()},
+            "path_roofline_ms": path_roof_ms, "path_roofline_frac": path_roof_ms / ms_step,
+            "cpu_baseline": cpu,
+            "e2e": {"value": c.num_q / (e2e_ms / 1000.0), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"], "samples": clocks["samples"]},
+            "dense_baseline": {"prefill_ms": dense_ms, "sparse_over_dense_speedup": dense_ms / ms_step,
+                               "dense_prefill_tflops": work["dense_flops"] / (dense_ms * 1e-3) / 1e12,
+                               "decode_us": dense_dec_ms * 1000,
+                               "decode_speedup": dense_dec_ms * 1000 / graph_us,
+                               "dense_decode_gbs": workd["dense_bytes_decode"] / (dense_dec_ms * 1e-3) / 1e9,
+                               "article_ratios_context": {"prefill": 7.6, "decode": 4.9}},
+            "decode": {"workload": cd.name, "us_per_step": graph_us, "cuda_graph": True,
+                       "us_per_step_eager": statistics.mean(dstep_ms) * 1000,
+                       "stages_us": {k: v["ms"] * 1000 for k, v in dstages.items()},
+                       "stages": dstages, "path_roofline_us": dpath_roof_us,
+                       "path_roofline_frac": dpath_roof_us / graph_us,
+                       "e2e": {"value": d_e2e_us, "unit": "us/step", "h2d_bytes_per_step": dh2d,
+                               "d2h_bytes_per_step": dd2h},
+                       "gpu_launches_per_step": 8},
+        }
+        print(json.dumps(line))
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

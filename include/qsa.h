@@ -1,0 +1,175 @@
+/*
+ * qsa.h -- C-ABI of libqsa, the B200 (sm_100a) Qwen Sparse Attention (QSA) layer.
+ *
+ * The layer, as described in the article "Qwen's million-token window has a 2,048-token
+ * keyhole" (cronfeed.work), section "A million-token window with a selective view": an indexer
+ * with four query heads and one shared key head averages its keys over 4-token micro-blocks,
+ * scores the micro-blocks, keeps the best 512 (a 2,048-token budget that is the same at any
+ * context length) together with the unfinished block at the tail of the sequence, maps them back
+ * to token positions and runs the core attention there only.  Section "Three speed claims, three
+ * different experiments" of the same article measures it against paged grouped-query attention
+ * in chunked prefill and in multi-token decode; the dense entry points below are that baseline.
+ *
+ * Readings this library takes where the article is silent (all configurable fields excepted):
+ *   k_b   = bf16_rne( (k[4b] + k[4b+1] + k[4b+2] + k[4b+3]) / 4 )   (computed exactly, then rounded)
+ *   s_b(t) = sum_{h=0..3} w_h(t) * max(0, q_h(t) . k_b)                 (bf16 operands, fp32 accum.)
+ *   candidates of query position t: blocks b < t / 4 (complete blocks not holding t);
+ *   selection: top topk_blocks candidates by (score desc, block asc), plus the tail block t / 4;
+ *   core attention of query head h uses key/value head h / (Hq / Hkv), softmax scale
+ *   1/sqrt(head_dim) unless set, fp32 online softmax, bf16 output (round to nearest even).
+ *
+ * Memory model.  Every buffer is caller-owned device memory unless marked "host"; the library
+ * allocates nothing and keeps no state beyond cached device attributes.  Every call is an
+ * asynchronous launch on `stream` (a cudaStream_t; NULL = legacy default stream) and returns
+ * after argument checks: QSA_OK, QSA_ERR_INVALID_ARG (bad sizes / NULL pointers / workspace too
+ * small is QSA_ERR_WORKSPACE), QSA_ERR_UNSUPPORTED (shape outside what the kernels are built for),
+ * or QSA_ERR_CUDA (a launch failed; cudaGetLastError() is cleared and folded into the status).
+ * Problems that are only visible in device data (a page id outside the pool, a position outside
+ * the page table, an out-of-range selection entry) never trap: the offending read is skipped or
+ * zero-filled and a QSA_DEVERR_* bit is OR-ed into *batch->err_flag, which the caller zeroes and
+ * reads after synchronising.
+ *
+ * Layouts (row-major, innermost last; bf16 = IEEE bfloat16 bit pattern):
+ *   q          bf16 [num_q, Hq, D]            core-attention queries (post positional encoding)
+ *   k_pool     bf16 [num_pages, 64, Hkv, D]   paged key cache; token p of sequence s lives in page
+ *   v_pool     bf16 [num_pages, 64, Hkv, D]     page_table[s][p / 64], slot p % 64
+ *   kcomp_pool bf16 [num_pages, 16, Di]       compressed indexer keys; block b of sequence s lives
+ *                                             in page page_table[s][b / 16], slot b % 16
+ *   idx_q      bf16 [num_q, 4, Di]            indexer queries;  idx_w bf16 [num_q, 4] head weights
+ *   sel        int32 [num_q, topk+1]          selected blocks, ascending, tail block last, -1 pad
+ *   n_sel      int32 [num_q]                  min(topk, t/4) + 1
+ */
+#ifndef QSA_H
+#define QSA_H
+#include <stddef.h>
+#include <stdint.h>
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* qsa_stream_t; /* same type as cudaStream_t */
+
+typedef enum qsa_status {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1,
+  QSA_ERR_UNSUPPORTED = 2,
+  QSA_ERR_WORKSPACE = 3,
+  QSA_ERR_CUDA = 4
+} qsa_status_t;
+
+/* Bits OR-ed into *err_flag by the kernels. */
+#define QSA_DEVERR_SEQ 1u      /* a sequence index outside [0, batch) */
+#define QSA_DEVERR_POS 2u      /* a position < 0 or beyond the page table */
+#define QSA_DEVERR_PAGE 4u     /* a page id outside [0, num_pages) */
+#define QSA_DEVERR_GROUP 8u    /* compress: a 4-row group is not one aligned block of one sequence */
+#define QSA_DEVERR_SEL 16u     /* attention: a selection entry outside [0, t/4] */
+#define QSA_DEVERR_TIMEOUT 32u /* a bounded wait inside a kernel gave up */
+#define QSA_DEVERR_INTERNAL 64u
+
+typedef enum qsa_op {
+  QSA_OP_INDEX_SCORE_TOPK = 1,
+  QSA_OP_SPARSE_ATTN_DECODE = 2,
+  QSA_OP_DENSE_ATTN_DECODE = 3
+} qsa_op_t;
+
+typedef struct qsa_config {
+  int32_t num_q_heads;  /* Hq, a multiple of num_kv_heads with Hq/Hkv in {1,2,4,8,16} */
+  int32_t num_kv_heads; /* Hkv in {1, 2, 4, 8} */
+  int32_t head_dim;     /* D in {64, 128} */
+  int32_t idx_heads;    /* Hi, must be 4 */
+  int32_t idx_dim;      /* Di in {32, 64, 128} */
+  int32_t block_tokens; /* must be 4 */
+  int32_t topk_blocks;  /* 1..512; the article's budget is 512 */
+  int32_t page_tokens;  /* must be 64 */
+  float softmax_scale;  /* <= 0 selects 1/sqrt(head_dim) */
+  int32_t score_path;   /* qsa_index_score_topk algorithm: 0 auto, 1 streaming, 2 materialised */
+} qsa_config_t;
+
+typedef struct qsa_batch {
+  int32_t batch;             /* host: number of sequences */
+  int32_t num_q;             /* host: number of query rows */
+  int32_t max_pages_per_seq; /* host: row length of page_table */
+  int32_t num_pages;         /* host: pages in each pool */
+  int32_t max_pos;           /* host: an upper bound on every q_pos (sizes grids/workspace) */
+  const int32_t* q_seq;      /* device [num_q]: sequence of each query row */
+  const int32_t* q_pos;      /* device [num_q]: absolute position t of each query row */
+  const int32_t* page_table; /* device [batch, max_pages_per_seq]: physical page ids */
+  int32_t* err_flag;         /* device [1]: QSA_DEVERR_* bits, zeroed by the caller */
+} qsa_batch_t;
+
+const char* qsa_status_string(qsa_status_t status);
+int32_t qsa_version(void);
+
+/* Bytes of workspace `op` needs for this batch (num_splits as passed to the call; 0 = auto).
+ * *bytes is written on QSA_OK.  The workspace is caller-owned device memory, at least 256-byte
+ * aligned, and may be reused between calls on the same stream. */
+qsa_status_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_batch_t* batch, qsa_op_t op,
+                                int32_t num_splits, size_t* bytes);
+
+/* Step (a), micro-block compression (article section "A million-token window with a selective
+ * view": keys are compressed four tokens at a time).  The n_new rows of idx_k (bf16 [n_new, Di])
+ * are the raw indexer keys of new tokens; n_new must be a multiple of 4 and rows 4j..4j+3 must
+ * be positions 4b..4b+3 of one sequence (new_seq / new_pos: device int32 [n_new]).  For each such
+ * group, kcomp_pool[page_table[s][b/16]][b%16] = bf16_rne(mean of the 4 rows), summed exactly.
+ * A malformed group is skipped and flagged QSA_DEVERR_GROUP.  batch->q_seq/q_pos are unused. */
+qsa_status_t qsa_index_compress(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                const void* idx_k, const int32_t* new_seq,
+                                const int32_t* new_pos, int32_t n_new, void* kcomp_pool,
+                                qsa_stream_t stream);
+
+/* Steps (b)+(c), indexer scoring and selection (same section: the indexer ranks the
+ * micro-blocks; a budget of 512 plus the unfinished tail block, per the article's opening).
+ * For every query row: scores of all candidate blocks b < t/4 of its sequence (kcomp_pool must
+ * hold them: compress runs first, including the blocks completed by this chunk), exact top
+ * topk_blocks by (score desc, block asc), plus the tail block t/4; written ascending to
+ * sel (int32 [num_q, topk+1], -1 padded), n_sel (int32 [num_q]) and, if not NULL, sel_scores
+ * (float [num_q, topk+1]: the fp32 score of each selected block, +INFINITY for the tail, NaN
+ * padding).  workspace: qsa_workspace_size(..., QSA_OP_INDEX_SCORE_TOPK, 0, ...) bytes. */
+qsa_status_t qsa_index_score_topk(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                  const void* idx_q, const void* idx_w, const void* kcomp_pool,
+                                  int32_t* sel, int32_t* n_sel, float* sel_scores,
+                                  void* workspace, size_t ws_bytes, qsa_stream_t stream);
+
+/* Diagnostic view of step (b): the fp32 score of every candidate block of every row, written to
+ * scores (float [num_q, ld]); entries b >= t/4 are left untouched.  ld >= max_pos/4. */
+qsa_status_t qsa_index_scores(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                              const void* idx_q, const void* idx_w, const void* kcomp_pool,
+                              float* scores, int64_t ld, qsa_stream_t stream);
+
+/* Steps (d)+(e), expansion and sparse core attention, prefill form (section "A million-token
+ * window with a selective view": core attention only at the selected positions).  Row i attends
+ * over positions {4b+j : b in sel[i][0..n_sel[i]), j < 4, 4b+j <= t} of its sequence, every query
+ * head sharing the row's selection.  out: bf16 [num_q, Hq, D]; lse: float [num_q, Hq] natural-log
+ * softmax normaliser, or NULL.  No workspace. */
+qsa_status_t qsa_sparse_attn_prefill(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                     const void* q, const void* k_pool, const void* v_pool,
+                                     const int32_t* sel, const int32_t* n_sel, void* out,
+                                     float* lse, qsa_stream_t stream);
+
+/* Same result as qsa_sparse_attn_prefill, computed split-K for few query rows (decode with
+ * multi-token prediction, section "Three speed claims, three different experiments"): each row's
+ * selected blocks are cut into num_splits pieces (0 = chosen from the device) processed in
+ * parallel, then merged by their log-sum-exp.  workspace: qsa_workspace_size(...,
+ * QSA_OP_SPARSE_ATTN_DECODE, num_splits, ...) bytes. */
+qsa_status_t qsa_sparse_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                    const void* q, const void* k_pool, const void* v_pool,
+                                    const int32_t* sel, const int32_t* n_sel, void* out,
+                                    float* lse, int32_t num_splits, void* workspace,
+                                    size_t ws_bytes, qsa_stream_t stream);
+
+/* The comparison baseline (section "Three speed claims, three different experiments": paged
+ * grouped-query attention): row i attends over every position 0..t of its sequence on the same
+ * pools.  Rows of one sequence should be contiguous (they share key/value tiles).  Prefill form:
+ * no workspace.  Decode form: split-K over the context with a log-sum-exp merge. */
+qsa_status_t qsa_dense_attn_prefill(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                    const void* q, const void* k_pool, const void* v_pool,
+                                    void* out, float* lse, qsa_stream_t stream);
+qsa_status_t qsa_dense_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                   const void* q, const void* k_pool, const void* v_pool,
+                                   void* out, float* lse, int32_t num_splits, void* workspace,
+                                   size_t ws_bytes, qsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

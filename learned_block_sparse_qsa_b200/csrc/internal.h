@@ -1,0 +1,53 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qsa.h"
+
+namespace qsa {
+
+struct Geometry {  // validated copy of the config + batch scalars
+  int Hq, Hkv, D, G, Di, topk, batch, num_q, max_pages, num_pages, max_pos;
+  float scale_log2;  // softmax scale * log2(e)
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  const int32_t* page_table;
+  int32_t* err;
+};
+
+int num_sms();
+
+// compress.cu
+cudaError_t launch_compress(const Geometry& g, const void* idx_k, const int32_t* new_seq,
+                            const int32_t* new_pos, int n_new, void* kcomp, cudaStream_t s);
+
+// score.cu
+size_t score_workspace_bytes(const Geometry& g, int path);
+int resolve_score_path(const Geometry& g, int requested);
+cudaError_t launch_score_topk(const Geometry& g, int path, const void* idx_q, const void* idx_w,
+                              const void* kcomp, int32_t* sel, int32_t* n_sel, float* sel_scores,
+                              void* ws, size_t ws_bytes, cudaStream_t s);
+cudaError_t launch_scores_only(const Geometry& g, const void* idx_q, const void* idx_w,
+                               const void* kcomp, float* scores, int64_t ld, cudaStream_t s);
+
+// attn.cu
+int resolve_sparse_splits(const Geometry& g, int requested);
+size_t sparse_decode_workspace_bytes(const Geometry& g, int splits);
+cudaError_t launch_sparse_attn(const Geometry& g, const void* q, const void* k_pool,
+                               const void* v_pool, const int32_t* sel, const int32_t* n_sel,
+                               int sel_stride, void* out, float* lse, int splits, void* ws,
+                               cudaStream_t s);
+
+// dense.cu
+int resolve_dense_splits(const Geometry& g, int requested);
+size_t dense_decode_workspace_bytes(const Geometry& g, int splits);
+cudaError_t launch_dense_attn(const Geometry& g, const void* q, const void* k_pool,
+                              const void* v_pool, void* out, float* lse, int splits, void* ws,
+                              cudaStream_t s);
+
+// combine (attn.cu): merge split partials [num_q, splits, Hq] of (o fp32 [D], lse2) -> bf16
+cudaError_t launch_combine(const Geometry& g, const float* part_o, const float* part_lse,
+                           int splits, void* out, float* lse, cudaStream_t s);
+
+}  // namespace qsa

@@ -1,0 +1,92 @@
+"""QsaRunner: one QSA layer step = the C-ABI calls in order, with cached workspaces.
+
+The steps, as the article "Qwen's million-token window has a 2,048-token keyhole" describes the
+layer (section "A million-token window with a selective view"): compress the new indexer keys
+into 4-token micro-blocks, score and select the best blocks plus the tail, then run core
+attention over the selected positions only.  Prefill uses the one-CTA-per-row attention; decode
+(few rows, section "Three speed claims, three different experiments") uses the split-K form.
+
+PyTorch only allocates the workspaces and the error flag; every step runs in libqsa's kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import (QSA_OP_DENSE_ATTN_DECODE, QSA_OP_INDEX_SCORE_TOPK, QSA_OP_SPARSE_ATTN_DECODE,
+               QsaBatch, QsaConfig, qsa_dense_attn_decode, qsa_dense_attn_prefill,
+               qsa_index_compress, qsa_index_score_topk, qsa_sparse_attn_decode,
+               qsa_sparse_attn_prefill, qsa_workspace_size)
+
+
+class QsaRunner:
+    def __init__(self, cfg: QsaConfig, device="cuda"):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self._ws: dict[int, torch.Tensor] = {}
+        self._keep = []
+
+    def batch(self, *, batch: int, num_q: int, max_pages: int, num_pages: int, max_pos: int,
+              q_seq: torch.Tensor, q_pos: torch.Tensor, page_table: torch.Tensor) -> QsaBatch:
+        self._keep = [q_seq, q_pos, page_table]
+        return QsaBatch(batch, num_q, max_pages, num_pages, max_pos, q_seq.data_ptr(),
+                        q_pos.data_ptr(), page_table.data_ptr(), self.err.data_ptr())
+
+    def workspace(self, b: QsaBatch, op: int, splits: int = 0):
+        n = qsa_workspace_size(self.cfg, b, op, splits)
+        buf = self._ws.get(op)
+        if n > 0 and (buf is None or buf.numel() < n):
+            buf = torch.empty(n, dtype=torch.uint8, device=self.device)
+            self._ws[op] = buf
+        return (buf if n > 0 else None), n
+
+    def compress(self, b: QsaBatch, idx_k_new, new_seq, new_pos, kcomp_pool, stream=None):
+        qsa_index_compress(self.cfg, b, idx_k_new, new_seq, new_pos, int(new_seq.numel()), kcomp_pool,
+                           stream)
+
+    def select(self, b: QsaBatch, idx_q, idx_w, kcomp_pool, sel, n_sel, sel_scores=None, stream=None):
+        ws, n = self.workspace(b, QSA_OP_INDEX_SCORE_TOPK)
+        qsa_index_score_topk(self.cfg, b, idx_q, idx_w, kcomp_pool, sel, n_sel, sel_scores, ws, n,
+                             stream)
+
+    def prefill(self, b: QsaBatch, *, q, idx_q, idx_w, kcomp_pool, k_pool, v_pool, out, sel, n_sel,
+                idx_k_new=None, new_seq=None, new_pos=None, lse=None, sel_scores=None, stream=None):
+        """Whole prefill step: compress (if new keys are given) -> score/select -> attention."""
+        if idx_k_new is not None:
+            self.compress(b, idx_k_new, new_seq, new_pos, kcomp_pool, stream)
+        self.select(b, idx_q, idx_w, kcomp_pool, sel, n_sel, sel_scores, stream)
+        qsa_sparse_attn_prefill(self.cfg, b, q, k_pool, v_pool, sel, n_sel, out, lse, stream)
+        return out
+
+    def decode(self, b: QsaBatch, *, q, idx_q, idx_w, kcomp_pool, k_pool, v_pool, out, sel, n_sel,
+               idx_k_new=None, new_seq=None, new_pos=None, lse=None, sel_scores=None, splits=0,
+               stream=None):
+        """Whole decode step: compress the new block -> score/select -> split-K attention."""
+        if idx_k_new is not None:
+            self.compress(b, idx_k_new, new_seq, new_pos, kcomp_pool, stream)
+        self.select(b, idx_q, idx_w, kcomp_pool, sel, n_sel, sel_scores, stream)
+        ws, n = self.workspace(b, QSA_OP_SPARSE_ATTN_DECODE, splits)
+        qsa_sparse_attn_decode(self.cfg, b, q, k_pool, v_pool, sel, n_sel, out, lse, splits, ws, n,
+                               stream)
+        return out
+
+    def dense(self, b: QsaBatch, *, q, k_pool, v_pool, out, lse=None, decode=False, splits=0,
+              stream=None):
+        """Dense paged-GQA baseline on the same pools."""
+        if decode:
+            ws, n = self.workspace(b, QSA_OP_DENSE_ATTN_DECODE, splits)
+            qsa_dense_attn_decode(self.cfg, b, q, k_pool, v_pool, out, lse, splits, ws, n, stream)
+        else:
+            qsa_dense_attn_prefill(self.cfg, b, q, k_pool, v_pool, out, lse, stream)
+        return out
+
+    def error_bits(self) -> int:
+        return int(self.err.item())
+
+    def clear_error(self):
+        self.err.zero_()
+
+
+__all__ = ["QsaRunner", "ctypes"]

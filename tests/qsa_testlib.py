@@ -1,0 +1,171 @@
+"""Helpers for the parity tests: run the CUDA path through the C-ABI binding, and compute the
+oracle's answer for the same seeded inputs on the host.  The two sides share only the input
+generator (qsa_synth); every expected value comes from oracle/."""
+from __future__ import annotations
+
+import functools
+import math
+
+import numpy as np
+
+from oracle import qsa_oracle as orc
+from qsa_synth import CONFIGS, Config, HostInputs
+
+# tolerances (attention allclose form; indexer scores relative to the row's k-th score)
+ATTN_ATOL, ATTN_RTOL = 2e-2, 1e-2
+SCORE_RTOL = 1e-3
+
+
+def qsa_config(c: Config, score_path: int = 0, topk: int | None = None):
+    from learned_block_sparse_qsa_b200 import QsaConfig
+
+    return QsaConfig.make(c.Hq, c.Hkv, c.D, c.Di, topk=c.topk if topk is None else topk, Hi=c.Hi,
+                          block=c.block, page=c.page, score_path=score_path)
+
+
+class Run:
+    """Device inputs + runner + outputs of one workload."""
+
+    def __init__(self, c: Config, integer=False, score_path=0, topk=None, device="cuda"):
+        import torch
+
+        from learned_block_sparse_qsa_b200 import QsaRunner
+        from qsa_synth.device import DeviceInputs
+
+        self.torch = torch
+        self.c = c if topk is None else c.replace(topk=topk)
+        self.di = DeviceInputs(self.c, integer, device)
+        self.cfg = qsa_config(self.c, score_path)
+        self.runner = QsaRunner(self.cfg, device)
+        d = self.di
+        self.b = self.runner.batch(batch=c.batch, num_q=c.num_q, max_pages=c.max_pages,
+                                   num_pages=c.num_pages, max_pos=c.ctx - 1, q_seq=d.q_seq,
+                                   q_pos=d.q_pos, page_table=d.page_table)
+        k1 = self.c.topk + 1
+        self.sel = torch.empty(c.num_q, k1, dtype=torch.int32, device=device)
+        self.n_sel = torch.empty(c.num_q, dtype=torch.int32, device=device)
+        self.sel_scores = torch.empty(c.num_q, k1, dtype=torch.float32, device=device)
+        self.out = torch.empty_like(d.q)
+        self.lse = torch.empty(c.num_q, c.Hq, dtype=torch.float32, device=device)
+        self.setup_prefix()
+
+    def setup_prefix(self):
+        """Compressed keys of every block before the step's new tokens (not part of the step)."""
+        from learned_block_sparse_qsa_b200 import QsaBatch
+
+        for s in range(self.c.batch):
+            rows, seq, pos = self.di.prefix_rows(s)
+            if rows.shape[0]:
+                self.runner.compress(self.b, rows, seq, pos, self.di.kcomp_pool)
+        self.torch.cuda.synchronize()
+        _ = QsaBatch
+
+    def step(self, decode=None, splits=0):
+        d = self.di
+        decode = (self.c.mode == "decode") if decode is None else decode
+        kw = dict(q=d.q, idx_q=d.idx_q, idx_w=d.idx_w, kcomp_pool=d.kcomp_pool, k_pool=d.k_pool,
+                  v_pool=d.v_pool, out=self.out, sel=self.sel, n_sel=self.n_sel, lse=self.lse,
+                  sel_scores=self.sel_scores, idx_k_new=d.idx_k_new, new_seq=d.new_seq,
+                  new_pos=d.new_pos)
+        if decode:
+            self.runner.decode(self.b, splits=splits, **kw)
+        else:
+            self.runner.prefill(self.b, **kw)
+        self.torch.cuda.synchronize()
+        return self
+
+    def numpy(self):
+        t = self.torch
+        return dict(sel=self.sel.cpu().numpy(), n_sel=self.n_sel.cpu().numpy(),
+                    sel_scores=self.sel_scores.cpu().numpy(),
+                    out=self.out.view(t.int16).cpu().numpy().view(np.uint16),
+                    lse=self.lse.cpu().numpy())
+
+
+@functools.lru_cache(maxsize=16)
+def host(c: Config, integer: bool) -> HostInputs:
+    return HostInputs(c, integer)
+
+
+@functools.lru_cache(maxsize=8)
+def host_kcomp(c: Config, integer: bool, s: int) -> np.ndarray:
+    """Oracle compression of every complete block of sequence s (bf16 bits [ctx//4, Di])."""
+    h = host(c, integer)
+    return orc.compress(h.idx_k(s, 0, c.ctx))
+
+
+def oracle_select_row(c: Config, integer: bool, r: int, topk: int | None = None):
+    """(sel, all candidate scores) of query row r, by the oracle."""
+    h = host(c, integer)
+    q_seq, q_pos = h.rows()
+    s, t = int(q_seq[r]), int(q_pos[r])
+    kc = host_kcomp(c, integer, s)
+    return orc.qsa_select(kc, h.idx_q([r])[0], h.idx_w([r])[0], t, c.topk if topk is None else topk)
+
+
+def oracle_attend_row(c: Config, integer: bool, r: int, sel: np.ndarray):
+    """Oracle attention of row r over the positions of the given selection."""
+    h = host(c, integer)
+    q_seq, q_pos = h.rows()
+    s, t = int(q_seq[r]), int(q_pos[r])
+    pos = orc.expand(np.asarray(sel), t)
+    k, v = h.kv(s, pos)
+    return orc.attend(h.q([r])[0], k, v)
+
+
+def oracle_dense_row(c: Config, integer: bool, r: int):
+    h = host(c, integer)
+    q_seq, q_pos = h.rows()
+    s, t = int(q_seq[r]), int(q_pos[r])
+    k, v = h.kv(s, np.arange(t + 1))
+    return orc.dense_causal(h.q([r])[0], k, v, t)
+
+
+def kth_score(scores: np.ndarray, k: int) -> float:
+    if scores.size == 0:
+        return 0.0
+    k = min(k, scores.size)
+    return float(np.partition(scores, scores.size - k)[scores.size - k])
+
+
+def check_selection(gsel_row, gn, gsc_row, ref_sel, ref_scores, t, topk, exact: bool):
+    """GPU selection of one row against the oracle's.  Exact mode (integer inputs): identical
+    blocks and identical fp32 scores.  Otherwise: same count and tail; every selected block's
+    score within SCORE_RTOL of the oracle's (relative to max(|s|, |s_k|)); blocks selected by only
+    one side must lie within SCORE_RTOL*|s_k| of the k-th score s_k."""
+    n = min(topk, t // 4) + 1
+    assert gn == n, (gn, n)
+    g = np.asarray(gsel_row[:n], dtype=np.int64)
+    assert g[-1] == t // 4 and np.all(np.diff(g) > 0), g
+    assert np.all(np.asarray(gsel_row[n:]) == -1)
+    gs = np.asarray(gsc_row[: n - 1], dtype=np.float64)
+    if exact:
+        assert np.array_equal(g, ref_sel), (g, ref_sel)
+        assert np.array_equal(gs, ref_scores[g[:-1]])
+        return 0
+    sk = kth_score(ref_scores, topk)
+    scale = np.maximum(np.abs(ref_scores[g[:-1]]), abs(sk)) + 1e-6
+    assert np.all(np.abs(gs - ref_scores[g[:-1]]) <= SCORE_RTOL * scale), "score mismatch"
+    a, b = set(g[:-1].tolist()), set(ref_sel[:-1].tolist())
+    diff = a ^ b
+    for blk in diff:
+        assert abs(ref_scores[blk] - sk) <= SCORE_RTOL * abs(sk) + 1e-6, (blk, ref_scores[blk], sk)
+    return len(diff)
+
+
+def check_attention(gout_row_bits, glse_row, ref_o, ref_lse):
+    go = orc.bf16_to_f64(gout_row_bits)
+    assert np.allclose(go, ref_o, atol=ATTN_ATOL, rtol=ATTN_RTOL), float(np.max(np.abs(go - ref_o)))
+    if glse_row is not None:
+        assert np.allclose(glse_row, ref_lse, atol=ATTN_ATOL, rtol=ATTN_RTOL)
+
+
+def sample_rows(c: Config, n: int) -> list[int]:
+    """Evenly spaced query rows including the first and the last."""
+    if c.num_q <= n:
+        return list(range(c.num_q))
+    return sorted(set(np.linspace(0, c.num_q - 1, n).round().astype(int).tolist()))
+
+
+__all__ = ["CONFIGS", "Run", "host_kcomp", "oracle_select_row", "oracle_attend_row",
+           "oracle_dense_row", "check_selection", "check_attention", "sample_rows", "math"]

@@ -1,0 +1,94 @@
+"""CPU checks of the C-ABI boundary: the libraries load, export every declared symbol, and the
+host-side argument checks answer with the documented status codes (no kernel is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared(header):
+    text = open(os.path.join(ROOT, "include", header)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:qsa|qsyn)_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.mark.parametrize("header,lib", [("qsa.h", "learned_block_sparse_qsa_b200/libqsa.so"),
+                                        ("qsa_synth.h", "qsa_synth/libqsa_synth.so")])
+def test_library_exports_every_declared_symbol(header, lib):
+    names = declared(header)
+    assert len(names) >= 2
+    so = ctypes.CDLL(os.path.join(ROOT, lib))
+    missing = [n for n in names if not hasattr(so, n)]
+    assert not missing, missing
+
+
+def test_qsa_header_declares_the_layer_entry_points():
+    names = declared("qsa.h")
+    for n in ["qsa_index_compress", "qsa_index_score_topk", "qsa_sparse_attn_prefill",
+              "qsa_sparse_attn_decode", "qsa_dense_attn_prefill", "qsa_dense_attn_decode",
+              "qsa_workspace_size", "qsa_status_string"]:
+        assert n in names
+
+
+import learned_block_sparse_qsa_b200 as q  # noqa: E402
+
+
+def mk_batch(num_q=16, batch=1, max_pages=4, num_pages=4, max_pos=255, ptr=0x1000):
+    return q.QsaBatch(batch, num_q, max_pages, num_pages, max_pos, ptr, ptr, ptr, ptr)
+
+
+def test_status_strings_and_version():
+    assert q.qsa_status_string(0) == "ok"
+    assert "workspace" in q.qsa_status_string(3)
+    assert q.qsa_version() >= 100
+
+
+def test_workspace_sizes_are_host_computable():
+    cfg = q.QsaConfig.make(32, 4, 128, 128)
+    b = mk_batch(num_q=16384, max_pages=16384, num_pages=16384, max_pos=1048575)
+    n_stream = q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK)
+    assert n_stream == 16384 * 2048 * 8           # streaming path: 2048 candidate slots per row
+    b = mk_batch(num_q=16, batch=4, max_pages=16384, num_pages=65536, max_pos=1048575)
+    n_mat = q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK)
+    assert n_mat >= 16 * 262144 * 12              # materialised path: scores + boundary keys
+    assert q.qsa_workspace_size(cfg, b, q.QSA_OP_SPARSE_ATTN_DECODE, 1) == 0
+    assert q.qsa_workspace_size(cfg, b, q.QSA_OP_SPARSE_ATTN_DECODE, 8) >= 16 * 8 * 32 * 129 * 4
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("block_tokens", 8, q.QSA_ERR_UNSUPPORTED), ("idx_heads", 2, q.QSA_ERR_UNSUPPORTED),
+    ("head_dim", 96, q.QSA_ERR_UNSUPPORTED), ("topk_blocks", 0, q.QSA_ERR_UNSUPPORTED),
+    ("topk_blocks", 513, q.QSA_ERR_UNSUPPORTED), ("num_q_heads", 6, q.QSA_ERR_INVALID_ARG),
+    ("page_tokens", 32, q.QSA_ERR_UNSUPPORTED), ("score_path", 3, q.QSA_ERR_INVALID_ARG)])
+def test_invalid_config_rejected_before_launch(field, value, status):
+    cfg = q.QsaConfig.make(32, 4, 128, 128)
+    setattr(cfg, field, value)
+    with pytest.raises(q.QsaError) as e:
+        q.qsa_workspace_size(cfg, mk_batch(), q.QSA_OP_INDEX_SCORE_TOPK)
+    assert e.value.status == status
+
+
+def test_invalid_arguments_rejected_before_launch():
+    cfg = q.QsaConfig.make(4, 1, 64, 32)
+    b = mk_batch()
+    with pytest.raises(q.QsaError) as e:   # n_new not a multiple of 4
+        q.qsa_index_compress(cfg, b, 0x1000, 0x1000, 0x1000, 6, 0x1000, stream=0)
+    assert e.value.status == q.QSA_ERR_INVALID_ARG
+    with pytest.raises(q.QsaError) as e:   # misaligned key pointer
+        q.qsa_index_compress(cfg, b, 0x1002, 0x1000, 0x1000, 8, 0x1000, stream=0)
+    assert e.value.status == q.QSA_ERR_INVALID_ARG
+    with pytest.raises(q.QsaError) as e:   # no workspace
+        q.qsa_index_score_topk(cfg, b, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0, stream=0)
+    assert e.value.status == q.QSA_ERR_WORKSPACE
+    with pytest.raises(q.QsaError) as e:   # missing page table
+        bad = mk_batch()
+        bad.page_table = None
+        q.qsa_sparse_attn_prefill(cfg, bad, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, stream=0)
+    assert e.value.status == q.QSA_ERR_INVALID_ARG
+    with pytest.raises(q.QsaError) as e:   # decode with splits but no workspace
+        q.qsa_sparse_attn_decode(cfg, b, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, 4,
+                                 None, 0, stream=0)
+    assert e.value.status == q.QSA_ERR_WORKSPACE
