@@ -40,6 +40,10 @@ DECODE = "C5"
 
 # ------------------------------------------------------------------------------------ helpers
 
+def log(msg: str):
+    print(f"[bench] {msg}", file=sys.stderr, flush=True)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -512,8 +516,12 @@ def main():
                 "traffic": traffic_for(ds["kernel_file"], f"{dom}@{PREFILL}")}
     path_roof_ms = (work["compress_bytes"] / (peaks["hbm"] * 1e9) + work["score_flops"] / (peaks["tf_sus"] * 1e12)
                     + work["attn_bytes"] / (peaks["hbm"] * 1e9)) * 1e3
+    log(f"prefill {c.name}: {ms_step:.3f} ms/step, {value / 1e6:.3f} M tok/s, stages "
+        + ", ".join(f"{k} {v['ms']:.3f} ms ({100 * v['frac']:.1f}% {v['bound']})" for k, v in stages.items()))
     e2e_ms, h2d, d2h = e2e_prefill(w, max(3, args.steps // 3), 2)
+    log(f"prefill e2e {e2e_ms:.3f} ms/step")
     dense_ms = dense_time_ms(w, False, 1)
+    log(f"dense prefill {dense_ms:.1f} ms ({work['dense_flops'] / (dense_ms * 1e-3) / 1e12:.1f} TFLOP/s)")
     del w
     torch.cuda.empty_cache()
 
@@ -523,10 +531,13 @@ def main():
     workd = algorithmic(cd, wd.q_pos_host)
     dsteps = max(50, 5 * args.steps)
     dstage_ms, dstep_ms, _ = time_steps(wd, True, dsteps, args.warmup, dist, flush=flush)
+    log("decode eager stages " + ", ".join(f"{k} {v * 1000:.1f} us" for k, v in dstage_ms.items()))
     graph_us, _ = graph_decode_us(wd, dsteps, args.warmup, flush)
+    log(f"decode graph {graph_us:.1f} us/step")
     graph_us = max_over_ranks(graph_us, dist)
     d_e2e_us, dh2d, dd2h = e2e_decode(wd, dsteps, args.warmup)
     dense_dec_ms = dense_time_ms(wd, True, 5, flush)
+    log(f"decode e2e {d_e2e_us:.1f} us/step; dense decode {dense_dec_ms * 1000:.1f} us")
     dstages = {
         "score_topk": dict(ms=dstage_ms["score_topk"], bound="hbm", unit="GB/s",
                            achieved=workd["score_bytes_decode"] / (dstage_ms["score_topk"] * 1e-3) / 1e9,

@@ -15,19 +15,31 @@ typedef __nv_bfloat16 bf16;
 // reported through the error flag instead of hanging the GPU.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
-// Opt a kernel into more than 48 KB of dynamic shared memory, once per device (host side).  Done
-// on the first launch so that later launches -- possibly inside a stream capture -- issue no
-// attribute calls.
-template <typename Kernel>
-inline cudaError_t set_smem_once(Kernel k, int bytes) {
-  static unsigned long long done = 0;  // bit d: set on device d
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per (kernel, device), on the
+// host.  Done at the first launch so that later launches -- possibly inside a stream capture --
+// issue no attribute calls.  Kernels are told apart by address (several share one signature).
+inline cudaError_t set_smem_once(const void* kernel, int bytes) {
+  struct Entry {
+    const void* k;
+    unsigned long long devs;
+  };
+  static Entry table[64];
+  static int used = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const unsigned long long bit = 1ull << (dev & 63);
-  if (done & bit) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done |= bit;
-  return e;
+  int i = 0;
+  while (i < used && table[i].k != kernel) ++i;
+  if (i < used && (table[i].devs & bit)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (i == used && used < 64) table[used++] = Entry{kernel, 0};
+  if (i < used) table[i].devs |= bit;
+  return cudaSuccess;
+}
+template <typename Kernel>
+inline cudaError_t set_smem_once(Kernel* k, int bytes) {
+  return set_smem_once(reinterpret_cast<const void*>(k), bytes);
 }
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
