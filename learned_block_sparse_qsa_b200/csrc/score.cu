@@ -22,76 +22,12 @@
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
+#include "score_common.cuh"
+
+#include <algorithm>
 
 namespace qsa {
 namespace {
-
-constexpr int kHi = 4;  // indexer query heads
-
-struct ScoreArgs {
-  const bf16* idx_q;  // [num_q, 4, DI]
-  const bf16* idx_w;  // [num_q, 4]
-  const bf16* kcomp;  // [num_pages, 16, DI]
-  const int32_t* q_seq;
-  const int32_t* q_pos;
-  const int32_t* page_table;
-  int num_q, batch, max_pages, num_pages, topk, max_pos;
-  int32_t* sel;
-  int32_t* n_sel;
-  float* sel_scores;
-  int sel_stride;
-  int32_t* err;
-};
-
-// Swizzled byte offset of 16-byte chunk `c` of row `r` in a [rows][DI] bf16 shared tile, chosen
-// so that ldmatrix over 8 consecutive rows touches 8 distinct bank groups.
-template <int DI>
-__device__ __forceinline__ uint32_t swz(int r, int c) {
-  if constexpr (DI >= 64) {
-    return (uint32_t)(r * (DI * 2) + ((c ^ (r & 7)) << 4));
-  } else {
-    return (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
-  }
-}
-
-// Validate a query row; returns its block limit t/4 (number of candidates) or -1.
-__device__ __forceinline__ int row_limit(const ScoreArgs& a, int r, int* seq_out) {
-  const int seq = a.q_seq[r];
-  const int pos = a.q_pos[r];
-  if (seq < 0 || seq >= a.batch) {
-    flag_error(a.err, QSA_DEVERR_SEQ);
-    return -1;
-  }
-  if (pos < 0 || pos / 64 >= a.max_pages || pos > a.max_pos) {
-    flag_error(a.err, QSA_DEVERR_POS);
-    return -1;
-  }
-  *seq_out = seq;
-  return pos / 4;
-}
-
-// cp.async one 64-block tile of sequence `seq`'s compressed keys into a swizzled [64][DI] tile.
-template <int DI, int NTHREADS>
-__device__ __forceinline__ void load_kcomp_tile(const ScoreArgs& a, int seq, int tile, int nb,
-                                                uint32_t dst) {
-  constexpr int CH = DI / 8;
-  for (int i = threadIdx.x; i < 64 * CH; i += NTHREADS) {
-    const int blk = i / CH, c = i % CH;
-    const int b = tile * 64 + blk;
-    bool valid = b < nb;
-    const bf16* src = a.kcomp;
-    if (valid) {
-      const int page = a.page_table[(long long)seq * a.max_pages + (b >> 4)];
-      if (page < 0 || page >= a.num_pages) {
-        if (c == 0) flag_error(a.err, QSA_DEVERR_PAGE);
-        valid = false;
-      } else {
-        src = a.kcomp + ((long long)page * 16 + (b & 15)) * DI + c * 8;
-      }
-    }
-    cp_async16(dst + swz<DI>(blk, c), src, valid);
-  }
-}
 
 // =============================================================================== streaming
 
@@ -120,7 +56,7 @@ struct StreamSmem {
 
 template <int DI>
 __global__ void __launch_bounds__(ST_THREADS, 2)
-    score_stream_kernel(ScoreArgs a, u64* __restrict__ cand, int cap) {
+    score_stream_kernel(ScoreArgs a, u64* __restrict__ cand, int cap, const int32_t* redo) {
   using S = StreamSmem<DI>;
   constexpr int CH = DI / 8;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -139,17 +75,28 @@ __global__ void __launch_bounds__(ST_THREADS, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row0 = blockIdx.x * ST_ROWS;
 
+  // redo != nullptr: only rows with redo[row] != 0 are computed (rows another kernel could not
+  // finish); every other row is left untouched.
   if (tid < ST_ROWS) {
     const int r = row0 + tid;
     int seq = -1, lim = -1;
-    if (r < a.num_q) lim = row_limit(a, r, &seq);
+    bool skip = false;
+    if (r < a.num_q) {
+      if (redo && redo[r] == 0) skip = true;
+      else lim = row_limit(a, r, &seq);
+    }
     sSeq[tid] = lim >= 0 ? seq : -1;
-    sPosv[tid] = lim;
+    sPosv[tid] = skip ? -2 : lim;
   }
   if (tid < 4) sMisc[tid] = 0;
   __syncthreads();
+  {
+    bool any = false;
+    for (int r = 0; r < ST_ROWS; ++r) any |= sSeq[r] >= 0;
+    if (!any && redo) return;  // nothing to redo in this tile (uniform over the CTA)
+  }
   for (int r = warp * 8; r < warp * 8 + 8; ++r)
-    if (row0 + r < a.num_q && sPosv[r] < 0)
+    if (row0 + r < a.num_q && sPosv[r] == -1)
       write_empty_selection(row0 + r, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
   for (int i = tid; i < ST_ROWS * kHi * CH; i += ST_THREADS) {
     const int row = i / (kHi * CH), h = (i / CH) % kHi, c = i % CH;
@@ -697,29 +644,6 @@ __global__ void __launch_bounds__(256) mat_final_kernel(ScoreArgs a, MatWs w) {
   }
 }
 
-ScoreArgs make_args(const Geometry& g, const void* idx_q, const void* idx_w, const void* kcomp,
-                    int32_t* sel, int32_t* n_sel, float* sel_scores) {
-  ScoreArgs a;
-  a.idx_q = static_cast<const bf16*>(idx_q);
-  a.idx_w = static_cast<const bf16*>(idx_w);
-  a.kcomp = static_cast<const bf16*>(kcomp);
-  a.q_seq = g.q_seq;
-  a.q_pos = g.q_pos;
-  a.page_table = g.page_table;
-  a.num_q = g.num_q;
-  a.batch = g.batch;
-  a.max_pages = g.max_pages;
-  a.num_pages = g.num_pages;
-  a.topk = g.topk;
-  a.max_pos = g.max_pos;
-  a.sel = sel;
-  a.n_sel = n_sel;
-  a.sel_scores = sel_scores;
-  a.sel_stride = g.topk + 1;
-  a.err = g.err;
-  return a;
-}
-
 long long mat_ld(const Geometry& g) { return ((long long)(g.max_pos / 4 + 1) + 63) / 64 * 64; }
 
 template <int DI>
@@ -741,12 +665,13 @@ cudaError_t run_dense_scores(const ScoreArgs& a, const Geometry& g, float* score
 }
 
 template <int DI>
-cudaError_t run_stream(const ScoreArgs& a, const Geometry& g, void* ws, cudaStream_t s) {
+cudaError_t run_stream(const ScoreArgs& a, const Geometry& g, void* ws, cudaStream_t s,
+                       const int32_t* redo = nullptr) {
   const int smem = StreamSmem<DI>::TOTAL;
   cudaError_t e = set_smem_once(score_stream_kernel<DI>, smem);
   if (e != cudaSuccess) return e;
   const int tiles = (g.num_q + ST_ROWS - 1) / ST_ROWS;
-  score_stream_kernel<DI><<<tiles, ST_THREADS, smem, s>>>(a, static_cast<u64*>(ws), stream_cap(g.topk));
+  score_stream_kernel<DI><<<tiles, ST_THREADS, smem, s>>>(a, static_cast<u64*>(ws), stream_cap(g.topk), redo);
   return cudaGetLastError();
 }
 
@@ -782,7 +707,11 @@ int resolve_score_path(const Geometry& g, int requested) {
 }
 
 size_t score_workspace_bytes(const Geometry& g, int path) {
-  if (path == 1) return (size_t)g.num_q * stream_cap(g.topk) * 8;
+  if (path == 1) {
+    size_t n = (size_t)g.num_q * stream_cap(g.topk) * 8;
+    if (score_tc_supported(g)) n = std::max(n, score_tc_workspace_bytes(g));
+    return n;
+  }
   return mat_bytes(g);
 }
 
@@ -793,6 +722,13 @@ cudaError_t launch_score_topk(const Geometry& g, int path, const void* idx_q, co
   if (g.num_q == 0) return cudaSuccess;
   const ScoreArgs a = make_args(g, idx_q, idx_w, kcomp, sel, n_sel, sel_scores);
   if (path == 1) {
+    if (score_tc_supported(g)) {
+      // tensor-core kernel first; the rows it flags are recomputed by the exact streaming kernel
+      int32_t* redo = nullptr;
+      cudaError_t e = launch_score_tc(a, g, ws, &redo, s);
+      if (e != cudaSuccess) return e;
+      return run_stream<128>(a, g, ws, s, redo);
+    }
     switch (g.Di) {
       case 32: return run_stream<32>(a, g, ws, s);
       case 64: return run_stream<64>(a, g, ws, s);

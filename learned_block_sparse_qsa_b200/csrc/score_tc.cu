@@ -1,0 +1,474 @@
+// Steps (b)+(c) on the 5th-generation tensor cores: indexer scoring with tcgen05.mma into TMEM,
+// fused with ReLU, head weighting, the causal limit and candidate filtering for the exact top-k.
+//
+// Article "Qwen's million-token window has a 2,048-token keyhole", section "A million-token window
+// with a selective view": four indexer query heads score every compressed micro-block of the one
+// shared key head and the best 512 are kept.  At a 1M-token context a 16,384-token prefill chunk is
+// a [65,536 x 128] x [128 x 262,144] bf16 contraction (4.4 TFLOP) whose 17 GB score matrix must
+// never be stored, so the selection is fused into the epilogue.
+//
+// CTA = 128 query rows (M = 128, one sequence segment at a time), warp-specialised:
+//   warp 0      TMA producer: the 4 heads' query tiles once (128 KB), then 64-block tiles of the
+//               compressed keys (4 pages x 2 K-halves of 16 rows x 128 B, 128-byte swizzle) into a
+//               4-stage ring;
+//   warp 1      owns the TMEM allocation (512 columns = two accumulator buffers x 4 heads x 64
+//               blocks) and one lane issues 4 x 8 tcgen05.mma (M=128, N=64, K=16) per tile;
+//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (= its 32 query rows) and half of
+//               the 64 columns; thread = (query row, column half).
+// Selection without in-loop compaction: the tile sequence is first every 16th tile (a sample),
+// then all tiles.  During the sample each thread keeps the 32 best sampled scores of its half-row
+// in registers; the row threshold tau = min over its two halves of the 32nd best, so about 1,024
+// of the row's scores are >= tau.  The full pass appends every (score >= tau, block) key to a
+// per-half-row buffer; the final step checks that at least min(512, t/4) keys were kept -- which
+// proves every true top-512 key was kept -- and selects exactly (radix select on 64-bit keys,
+// lower block index wins ties).  Rows that fail the check (adversarial score orders) or overflow
+// the buffer are recomputed by the exact streaming kernel, so the result never depends on the
+// sample.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "score_common.cuh"
+#include "select.cuh"
+
+namespace qsa {
+namespace {
+
+constexpr int TC_ROWS = 128;
+constexpr int TC_BLK = 64;      // blocks per tile (MMA N)
+constexpr int TC_NST = 4;       // compressed-key stages
+constexpr int TC_SAMPLE = 16;   // every 16th tile is sampled
+constexpr int TC_EPI = 8;       // epilogue warps
+constexpr int TC_THREADS = (2 + TC_EPI) * 32;
+constexpr int TC_A_BYTES = 4 * 2 * TC_ROWS * 128;  // 4 heads x 2 K-halves x 128 rows x 128 B
+constexpr int TC_B_STAGE = 2 * TC_BLK * 128;       // 2 K-halves x 64 rows x 128 B
+constexpr int TC_B_BYTES = TC_NST * TC_B_STAGE;
+constexpr int TC_SCRATCH_KEYS = TC_B_BYTES / TC_EPI / 8;  // 1024 keys per epilogue warp
+constexpr int TC_CAP = 2048;    // candidate slots per half-row
+
+struct TcMisc {
+  uint64_t full[TC_NST], empty[TC_NST], tfull[2], tempty[2], aload, mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+  int issued, consumed;  // B tiles issued by the producer / waited for by the MMA issuer
+  int seg, nb;
+  int lim[TC_ROWS];
+  int seq[TC_ROWS];
+  int cnt[2][TC_ROWS];
+  float thr[2][TC_ROWS];
+  float w[TC_ROWS][4];
+  uint32_t hist[TC_EPI][256];
+};
+constexpr int TC_SMEM = 1024 + TC_A_BYTES + TC_B_BYTES + (int)((sizeof(TcMisc) + 127) / 128 * 128);
+
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  uint64_t d = (uint64_t)((addr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;            // leading byte offset (unused with the 128-byte swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: 8 rows x 128 B
+  d |= (uint64_t)1 << 46;            // descriptor version
+  d |= (uint64_t)2 << 61;            // 128-byte swizzle
+  return d;
+}
+// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M=128, N=64.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_BLK >> 3) << 17) |
+                            ((uint32_t)(TC_ROWS >> 4) << 24);
+
+__device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* m, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+      "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma3d(uint32_t dst, const CUtensorMap* m, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),
+      "l"((uint64_t)m), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                   smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(TC_EPI * 32)); }
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    score_tc_kernel(ScoreArgs a, const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB, u64* __restrict__ cand,
+                    int32_t* __restrict__ redo) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + TC_A_BYTES;
+  TcMisc* m = reinterpret_cast<TcMisc*>(sB + TC_B_BYTES);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row0 = blockIdx.x * TC_ROWS;
+
+  if (tid == 0) {
+    for (int s = 0; s < TC_NST; ++s) {
+      mbar_init(&m->full[s], 1);
+      mbar_init(&m->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&m->tfull[b], 1);
+      mbar_init(&m->tempty[b], TC_EPI);
+    }
+    mbar_init(&m->aload, 1);
+    mbar_init(&m->mma_done, 1);
+    m->abort_flag = 0;
+    m->issued = 0;
+    m->consumed = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;\n" ::"r"(
+        smem_addr(&m->tmem_base)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+  }
+  if (tid < TC_ROWS) {
+    const int r = row0 + tid;
+    int seq = -1, lim = -1;
+    if (r < a.num_q) {
+      lim = row_limit(a, r, &seq);
+      redo[r] = 0;
+    }
+    m->seq[tid] = lim >= 0 ? seq : -1;
+    m->lim[tid] = lim;
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      m->w[tid][h] = r < a.num_q ? __bfloat162float(a.idx_w[(long long)r * kHi + h]) : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = m->tmem_base;
+  if (warp >= 2) {  // rows that failed validation get an empty selection
+    for (int r = (warp - 2) * 16; r < (warp - 2) * 16 + 16; ++r)
+      if (row0 + r < a.num_q && m->lim[r] < 0)
+        write_empty_selection(row0 + r, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
+  }
+
+  int it_base = 0;  // tiles of earlier segments (all roles count the same tiles)
+  bool first = true;
+  for (;;) {
+    __syncthreads();
+    if (tid == 0) {
+      int seg = -1, nb = 0;
+      for (int r = 0; r < TC_ROWS; ++r)
+        if (m->seq[r] >= 0) { seg = m->seq[r]; break; }
+      if (seg >= 0)
+        for (int r = 0; r < TC_ROWS; ++r)
+          if (m->seq[r] == seg) nb = max(nb, m->lim[r]);
+      m->seg = seg;
+      m->nb = nb;
+    }
+    __syncthreads();
+    const int seg = m->seg;
+    if (seg < 0 || m->abort_flag) break;
+    const int ntile = (m->nb + TC_BLK - 1) / TC_BLK;
+    const int nsamp = (ntile + TC_SAMPLE - 1) / TC_SAMPLE;
+    const int L = ntile > 0 ? nsamp + ntile : 0;
+
+    if (warp == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        if (first) {
+          mbar_arrive_expect_tx(&m->aload, TC_A_BYTES);
+          for (int h = 0; h < 4; ++h)
+            for (int at = 0; at < 2; ++at)
+              tma3d(smem_addr(sA + (h * 2 + at) * (TC_ROWS * 128)), &tmA, at * 64, h, row0, &m->aload);
+        }
+        const int32_t* pt = a.page_table + (long long)seg * a.max_pages;
+        for (int i = 0; i < L; ++i) {
+          const int gi = it_base + i;
+          const int s = gi % TC_NST;
+          if (gi >= TC_NST && !mbar_wait(&m->empty[s], ((gi / TC_NST) & 1) ^ 1, a.err)) {
+            m->abort_flag = 1;
+            break;
+          }
+          const int tile = i < nsamp ? i * TC_SAMPLE : i - nsamp;
+          mbar_arrive_expect_tx(&m->full[s], TC_B_STAGE);
+          for (int pg = 0; pg < 4; ++pg) {
+            const int lp = tile * 4 + pg;
+            int page = 0;  // pages past the table hold only masked blocks; page 0 keeps the copy in bounds
+            if (lp < a.max_pages) {
+              const int p = pt[lp];
+              if (p >= 0 && p < a.num_pages) page = p;
+              else flag_error(a.err, QSA_DEVERR_PAGE);
+            }
+            for (int at = 0; at < 2; ++at)
+              tma2d(smem_addr(sB + s * TC_B_STAGE + at * (TC_BLK * 128) + pg * 2048), &tmB, at * 64,
+                    page * 16, &m->full[s]);
+          }
+          m->issued = gi + 1;
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        bool ok = true;
+        if (first) ok = mbar_wait(&m->aload, 0, a.err);
+        for (int i = 0; ok && i < L; ++i) {
+          const int gi = it_base + i;
+          const int s = gi % TC_NST;
+          const int buf = gi & 1;
+          if (!mbar_wait(&m->full[s], (gi / TC_NST) & 1, a.err)) { ok = false; break; }
+          m->consumed = gi + 1;
+          if (gi >= 2 && !mbar_wait(&m->tempty[buf], ((gi >> 1) & 1) ^ 1, a.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t bst = smem_addr(sB + s * TC_B_STAGE);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const uint32_t ast = smem_addr(sA + h * 2 * (TC_ROWS * 128));
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint64_t ad = sw128_desc(ast + (ks >> 2) * (TC_ROWS * 128) + (ks & 3) * 32);
+              const uint64_t bd = sw128_desc(bst + (ks >> 2) * (TC_BLK * 128) + (ks & 3) * 32);
+              mma_f16(tbase + buf * 256 + h * TC_BLK, ad, bd, ks > 0 ? 1u : 0u);
+            }
+          }
+          mma_commit(&m->empty[s]);
+          mma_commit(&m->tfull[buf]);
+        }
+        if (!ok) m->abort_flag = 1;
+      }
+    } else {
+      // ---------------------------------------------------------------- epilogue
+      const int q = warp & 3;
+      const int hf = (warp - 2) >> 2;
+      const int row = q * 32 + lane;
+      const int lim = (m->seq[row] == seg) ? m->lim[row] : -1;
+      float w[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) w[h] = m->w[row][h];
+      float top[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) top[k] = -INFINITY;
+      float mn = -INFINITY, tau = -INFINITY;
+      int cnt = 0;
+      u64* mybuf = cand + ((long long)(row0 + row) * 2 + hf) * TC_CAP;
+      const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16);
+      bool dead = false;
+      for (int i = 0; i < L; ++i) {
+        const int gi = it_base + i;
+        const int buf = gi & 1;
+        if (i == nsamp) {  // end of the sample: fix the row threshold (every epilogue warp arrives)
+          m->thr[hf][row] = (lim > a.topk) ? mn : -INFINITY;
+          epi_sync();
+          tau = fminf(m->thr[0][row], m->thr[1][row]);
+        }
+        if (dead) continue;
+        if (!mbar_wait(&m->tfull[buf], (gi >> 1) & 1, a.err)) {
+          m->abort_flag = 1;
+          dead = true;
+          continue;
+        }
+        tc_fence_after();
+        const bool sample = i < nsamp;
+        const int tile = sample ? i * TC_SAMPLE : i - nsamp;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float v0[16], v1[16], v2[16], v3[16];
+          const uint32_t col = tl + buf * 256 + hf * 32 + c * 16;
+          tmem_ld16(col + 0 * TC_BLK, v0);
+          tmem_ld16(col + 1 * TC_BLK, v1);
+          tmem_ld16(col + 2 * TC_BLK, v2);
+          tmem_ld16(col + 3 * TC_BLK, v3);
+          tmem_wait_ld();
+          const int bbase = tile * TC_BLK + hf * 32 + c * 16;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float s = w[0] * fmaxf(v0[j], 0.f);
+            s = fmaf(w[1], fmaxf(v1[j], 0.f), s);
+            s = fmaf(w[2], fmaxf(v2[j], 0.f), s);
+            s = fmaf(w[3], fmaxf(v3[j], 0.f), s);
+            const int b = bbase + j;
+            if (b < lim) {
+              if (sample) {
+                if (s > mn) {  // replace one current minimum, then recompute the minimum
+                  bool done = false;
+#pragma unroll
+                  for (int k = 0; k < 32; ++k) {
+                    const bool hit = !done && top[k] == mn;
+                    top[k] = hit ? s : top[k];
+                    done |= hit;
+                  }
+                  mn = top[0];
+#pragma unroll
+                  for (int k = 1; k < 32; ++k) mn = fminf(mn, top[k]);
+                }
+              } else if (s >= tau) {
+                if (cnt < TC_CAP) mybuf[cnt] = make_key(s, (uint32_t)b);
+                ++cnt;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&m->tempty[buf]);
+      }
+      m->cnt[hf][row] = cnt;
+    }
+    __syncthreads();  // the segment's tiles are all consumed; stage memory is free
+
+    if (warp >= 2 && !m->abort_flag) {
+      // ---------------------------------------------------------------- exact final selection
+      const int e = warp - 2;
+      u64* scratch = reinterpret_cast<u64*>(sB) + e * TC_SCRATCH_KEYS;
+      uint32_t* sblk = reinterpret_cast<uint32_t*>(scratch);
+      float* ssc = reinterpret_cast<float*>(sblk + 512);
+      for (int rr = 0; rr < 16; ++rr) {
+        const int row = e * 16 + rr;
+        if (m->seq[row] != seg) continue;
+        const int lim = m->lim[row];
+        const int need = min(a.topk, lim);
+        const int n0 = m->cnt[0][row], n1 = m->cnt[1][row];
+        if (n0 > TC_CAP || n1 > TC_CAP || n0 + n1 < need) {
+          if (lane == 0) redo[row0 + row] = 1;
+          continue;
+        }
+        const u64* rb = cand + (long long)(row0 + row) * 2 * TC_CAP;
+        const int n = n0 + n1;
+        if (need > 0) {
+          u64* keys;
+          if (n <= TC_SCRATCH_KEYS) {
+            for (int i = lane; i < n; i += 32) scratch[i] = i < n0 ? rb[i] : rb[TC_CAP + i - n0];
+            keys = scratch;
+          } else {  // rare: pack both halves in place in global memory
+            u64* w = const_cast<u64*>(rb);
+            for (int base = 0; base < n1; base += 32) {
+              const int i = base + lane;
+              const u64 k = i < n1 ? w[TC_CAP + i] : 0ull;
+              __syncwarp();
+              if (i < n1) w[n0 + i] = k;
+              __syncwarp();
+            }
+            keys = w;
+          }
+          __syncwarp();
+          if (n > need) warp_select_compact(keys, n, need, m->hist[e]);
+          __syncwarp();
+          u64 kk[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) kk[u] = (lane + 32 * u) < need ? keys[lane + 32 * u] : 0ull;
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int i = lane + 32 * u;
+            if (i < need) {
+              sblk[i] = key_block(kk[u]);
+              ssc[i] = key_score(kk[u]);
+            }
+          }
+          __syncwarp();
+          warp_sort_blocks(sblk, ssc, need);
+        }
+        write_selection(row0 + row, need, lim, sblk, ssc, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    if (tid < TC_ROWS && m->seq[tid] == seg) m->seq[tid] = -1;
+    it_base += L;
+    first = false;
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncthreads();
+  if (m->abort_flag && warp == 0 && lane == 0) {  // let copies still in flight land first
+    mbar_wait(&m->aload, 0, a.err);
+    for (int gi = m->consumed; gi < m->issued; ++gi)
+      mbar_wait(&m->full[gi % TC_NST], (gi / TC_NST) & 1, a.err);
+  }
+  if (warp == 1) {
+    if (lane == 0 && it_base > 0) {  // every issued MMA has completed before TMEM is released
+      mma_commit(&m->mma_done);
+      mbar_wait(&m->mma_done, 0, a.err);
+    }
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;\n" ::"r"(tbase));
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool score_tc_supported(const Geometry& g) { return g.Di == 128 && encode_fn() != nullptr; }
+
+size_t score_tc_workspace_bytes(const Geometry& g) {
+  return (size_t)g.num_q * 2 * TC_CAP * 8 + ((size_t)g.num_q * 4 + 255) / 256 * 256;
+}
+
+// Launch the tensor-core kernel; rows it could not settle are flagged in `redo` (a workspace
+// slice) for the exact streaming kernel, which the caller launches next.
+cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int32_t** redo_out,
+                            cudaStream_t s) {
+  auto enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  u64* cand = static_cast<u64*>(ws);
+  int32_t* redo = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + (size_t)g.num_q * 2 * TC_CAP * 8);
+  *redo_out = redo;
+  CUtensorMap tmA, tmB;
+  {
+    cuuint64_t dims[3] = {128, 4, (cuuint64_t)g.num_q};
+    cuuint64_t strides[2] = {256, 1024};
+    cuuint32_t box[3] = {64, 1, TC_ROWS};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<bf16*>(a.idx_q), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    cuuint64_t dims[2] = {128, (cuuint64_t)g.num_pages * 16};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, 16};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<bf16*>(a.kcomp), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = set_smem_once(score_tc_kernel, TC_SMEM);
+  if (e != cudaSuccess) return e;
+  const int tiles = (g.num_q + TC_ROWS - 1) / TC_ROWS;
+  score_tc_kernel<<<tiles, TC_THREADS, TC_SMEM, s>>>(a, tmA, tmB, cand, redo);
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

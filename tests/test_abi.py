@@ -50,7 +50,7 @@ def test_workspace_sizes_are_host_computable():
     cfg = q.QsaConfig.make(32, 4, 128, 128)
     b = mk_batch(num_q=16384, max_pages=16384, num_pages=16384, max_pos=1048575)
     n_stream = q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK)
-    assert n_stream == 16384 * 2048 * 8           # streaming path: 2048 candidate slots per row
+    assert n_stream >= 16384 * 2048 * 8           # streaming path: >= 2048 candidate slots per row
     b = mk_batch(num_q=16, batch=4, max_pages=16384, num_pages=65536, max_pos=1048575)
     n_mat = q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK)
     assert n_mat >= 16 * 262144 * 12              # materialised path: scores + boundary keys

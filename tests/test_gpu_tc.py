@@ -1,0 +1,93 @@
+"""GPU parity of the tensor-core (tcgen05) indexer path: exact on integer inputs, ragged multi-
+sequence row tiles, and the exact fallback for rows whose sampled threshold keeps too few keys."""
+import numpy as np
+import pytest
+
+from oracle import qsa_oracle as orc
+from qsa_synth import Config
+from tests.qsa_testlib import Run, check_attention, check_selection, host, host_kcomp, score_bound
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+TC_PREFILL = Config("tc_prefill_T8192_di128", "prefill", 1, 8192, 8192, 8, 2, 64, 4, 128, seed=0x7C01)
+
+
+def check_rows(run, rows, integer, topk=None):
+    o = run.numpy()
+    c = run.c
+    topk = c.topk if topk is None else topk
+    h = host(c, integer)
+    q_seq, q_pos = h.rows()
+    for r in rows:
+        s, t = int(q_seq[r]), int(q_pos[r])
+        kc = host_kcomp(c, integer, s)
+        iq, iw = h.idx_q([r])[0], h.idx_w([r])[0]
+        ref_sel, ref_s = orc.qsa_select(kc, iq, iw, t, topk)
+        check_selection(o["sel"][r], o["n_sel"][r], o["sel_scores"][r], ref_sel, ref_s, t, topk,
+                        integer, score_bound(kc, iq, iw, t // 4))
+    return o
+
+
+def test_tc_prefill_integer_exact_all_rows():
+    run = Run(TC_PREFILL, integer=True, score_path=1).step()
+    check_rows(run, range(TC_PREFILL.num_q), True)
+    assert run.runner.error_bits() == 0
+
+
+def test_tc_prefill_random_sampled_rows_and_attention():
+    run = Run(TC_PREFILL, integer=False, score_path=1).step()
+    rows = list(range(0, 8192, 97)) + [8191]
+    o = check_rows(run, rows, False)
+    h = host(run.c, False)
+    _, q_pos = h.rows()
+    for r in rows[::4]:
+        t = int(q_pos[r])
+        n = o["n_sel"][r]
+        ref_o, ref_lse = orc.attend(h.q([r])[0], *h.kv(0, orc.expand(o["sel"][r][:n], t)))
+        check_attention(o["out"][r], o["lse"][r], ref_o, ref_lse)
+
+
+def test_tc_two_sequences_in_one_row_tile():
+    c = Config("tc_ragged_b3", "prefill", 3, 4096, 100, 8, 2, 64, 4, 128, shuffle_pages=True, seed=0x7C02)
+    run = Run(c, integer=True, score_path=1).step()
+    check_rows(run, range(c.num_q), True)
+
+
+def test_tc_small_budget_exact():
+    run = Run(TC_PREFILL.replace(ctx=3000, n_new=3000), integer=True, score_path=1, topk=37).step()
+    check_rows(run, range(0, 3000, 7), True, topk=37)
+
+
+def test_tc_fallback_on_decreasing_scores():
+    """Scores that fall with the block index defeat the sampled threshold (the sample's best blocks
+    are the first ones), so rows go to the exact fallback -- the result must still be exact."""
+    c = TC_PREFILL.replace(ctx=4096, n_new=4096)
+    run = Run(c, integer=True, score_path=1)
+    nb = c.ctx // 4
+    vals = np.zeros((c.ctx, c.Di), dtype=np.float32)
+    blk = np.arange(c.ctx) // 4
+    vals[:, 0] = (nb - blk) // 256
+    vals[:, 1] = (nb - blk) % 256
+    kbits = torch.tensor(vals).to(torch.bfloat16)
+    run.di.idx_k[0] = kbits.cuda()
+    run.di.idx_k_new.copy_(run.di.idx_k[0])
+    q = np.zeros((c.num_q, 4, c.Di), dtype=np.float32)
+    q[:, :, 0] = 256
+    q[:, :, 1] = 1
+    run.di.idx_q.copy_(torch.tensor(q).to(torch.bfloat16).cuda())
+    run.di.idx_w.fill_(1.0)
+    run.step()
+    o = run.numpy()
+    kc = orc.compress(kbits.view(torch.int16).numpy().view(np.uint16))
+    qb = torch.tensor(q[0]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    wb = torch.ones(4).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    _, q_pos = host(c, True).rows()
+    for r in list(range(0, c.num_q, 11)) + [c.num_q - 1]:
+        t = int(q_pos[r])
+        ref_sel, ref_s = orc.qsa_select(kc, qb, wb, t, c.topk)
+        check_selection(o["sel"][r], o["n_sel"][r], o["sel_scores"][r], ref_sel, ref_s, t, c.topk, True)
+        if t // 4 > 512:
+            assert list(ref_sel[:-1]) == list(range(512))  # the earliest blocks win
