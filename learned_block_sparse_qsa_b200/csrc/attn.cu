@@ -335,6 +335,307 @@ __global__ void __launch_bounds__(AttnCfg<D, HKV>::THREADS, 1) sparse_attn_kerne
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Swap-AB form for Hq/Hkv <= 8 (the article's 32 query heads over 4 KV heads): positions are the
+// M=16 rows of mma.m16n8k16 and the (up to) 8 query heads of a KV head are N=8, so no MMA row is
+// padding; P is transposed in registers with movmatrix for the P*V product, which computes O^T
+// (head dims x heads).  The producer first turns the CTA's whole slice of the selection into
+// physical row bases in shared memory (one pass, all lanes), so no dependent global load sits
+// between two stage issues.
+
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+constexpr int kMaxSel = 520;  // >= topk + 1
+// Consumer warps per KV head; a stage holds 4 blocks (16 positions) per consumer warp, so fewer
+// slices mean smaller stages and more of the shared-memory ring in flight.
+template <int HKV>
+constexpr int kSwSlices = HKV >= 4 ? 2 : 8 / HKV;
+
+template <int D, int HKV, int SLC>
+struct SwCfg {
+  static constexpr int NSLC = SLC;          // consumer warps per KV head
+  static constexpr int NCW = HKV * SLC;
+  static constexpr int NBS = 4 * NSLC;      // blocks per stage: 4 (= one 16-position chunk) per slice
+  static constexpr int ROWB = HKV * D * 2;  // one position row, all KV heads
+  static constexpr int BLKB = 4 * ROWB;     // one block: 4 contiguous rows
+  static constexpr int BPITCH = BLKB + 16;  // block slots skewed by 16 bytes
+  static constexpr int KVB = NBS * BPITCH;
+  static constexpr int STAGE = 2 * KVB;
+  static constexpr int NST = (200 * 1024) / STAGE > 8 ? 8 : (200 * 1024) / STAGE;
+  static constexpr int MERGE = NCW * (8 * D + 16) * 4;
+  static constexpr int BIG = (NST * STAGE > MERGE) ? NST * STAGE : MERGE;
+  static constexpr int POS_OFF = BIG;
+  static constexpr int ROW_OFF = POS_OFF + NST * NBS * 4 * 4;
+  static constexpr int BLK_OFF = ROW_OFF + kMaxSel * 4;
+  static constexpr int BAR_OFF = BLK_OFF + kMaxSel * 4;
+  static constexpr int TOTAL = BAR_OFF + 2 * NST * 8 + 16;
+  static constexpr int THREADS = (NCW + 1) * 32;
+  static_assert(NBS <= 32, "one producer lane per block slot");
+};
+
+// Stage layout: block slot j (0..NBS-1) holds the 4 rows of one selected block, K at
+// j*BPITCH and V at KVB + j*BPITCH.  Consumer warp `slc` owns slots 4*slc .. 4*slc+3; its MMA row
+// r (0..15) is row r>>2 of slot 4*slc + (r&3), so an 8-row ldmatrix reads 4 slots (distinct 16-byte
+// skews) x 2 rows: at most a 2-way bank conflict, while every full block arrives in one 4 KB copy.
+template <int D, int HKV, int SLC>
+__global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw_kernel(AttnArgs a) {
+  using C = SwCfg<D, HKV, SLC>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  int* sPos = reinterpret_cast<int*>(smem + C::POS_OFF);  // [stage][slot*4 + row-in-block]
+  int* sRow = reinterpret_cast<int*>(smem + C::ROW_OFF);  // page*64 + (b%16)*4, or -1
+  int* sBlk = reinterpret_cast<int*>(smem + C::BLK_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* empty = full + C::NST;
+  const uint32_t sbase = smem_addr(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.x, split = blockIdx.y;
+
+  const int seq = a.q_seq[row];
+  const int t = a.q_pos[row];
+  const bool ok = seq >= 0 && seq < a.batch && t >= 0 && t / 64 < a.max_pages;
+  int n = ok ? a.n_sel[row] : 0;
+  if (n < 0 || n > a.sel_stride || n > kMaxSel) {
+    if (tid == 0) flag_error(a.err, QSA_DEVERR_SEL);
+    n = max(0, min(min(n, a.sel_stride), kMaxSel));
+  }
+  if (!ok && tid == 0) flag_error(a.err, (seq < 0 || seq >= a.batch) ? QSA_DEVERR_SEQ : QSA_DEVERR_POS);
+  const int blo = (int)((long long)n * split / a.splits);
+  const int bhi = (int)((long long)n * (split + 1) / a.splits);
+  const int nblk = bhi - blo;
+  const int nstages = (nblk + C::NBS - 1) / C::NBS;
+
+  if (tid == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::NCW);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == C::NCW) {
+    // ================================================================ producer
+    const int32_t* selrow = a.sel + (long long)row * a.sel_stride;
+    const int32_t* ptab = a.page_table + (long long)(ok ? seq : 0) * a.max_pages;
+    for (int i = lane; i < nblk; i += 32) {  // selection slice -> physical row bases
+      const int b = selrow[blo + i];
+      int rb = -1;
+      if (b < 0 || b > t / 4) {
+        flag_error(a.err, QSA_DEVERR_SEL);
+      } else {
+        const int page = ptab[b >> 4];
+        if (page < 0 || page >= a.num_pages) flag_error(a.err, QSA_DEVERR_PAGE);
+        else rb = page * 64 + (b & 15) * 4;
+      }
+      sRow[i] = rb;
+      sBlk[i] = b;
+    }
+    __syncwarp();
+    for (int it = 0; it < nstages; ++it) {
+      const int st = it % C::NST;
+      if (it >= C::NST && !mbar_wait(&empty[st], ((it / C::NST) - 1) & 1, a.err)) break;
+      const uint32_t kdst = sbase + st * C::STAGE + lane * C::BPITCH;
+      const uint32_t vdst = kdst + C::KVB;
+      // lane j < NBS serves block slot j: rows valid = 4 (whole block), 1..3 (tail), or 0
+      int nvalid = 0, rb = -1;
+      if (lane < C::NBS) {
+        const int i = it * C::NBS + lane;
+        int b = 0;
+        if (i < nblk && sRow[i] >= 0) {
+          rb = sRow[i];
+          b = sBlk[i];
+          nvalid = min(4, t - 4 * b + 1);
+        }
+        int* pp = sPos + (st * C::NBS + lane) * 4;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          pp[r] = r < nvalid ? 4 * b + r : -1;
+          if (r >= nvalid) {  // masked row: zeros keep 0 * V finite
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            uint4* kz = reinterpret_cast<uint4*>(smem + st * C::STAGE + lane * C::BPITCH + r * C::ROWB);
+            uint4* vz = reinterpret_cast<uint4*>(smem + st * C::STAGE + C::KVB + lane * C::BPITCH + r * C::ROWB);
+#pragma unroll 4
+            for (int j = 0; j < C::ROWB / 16; ++j) {
+              kz[j] = z;
+              vz[j] = z;
+            }
+          }
+        }
+      }
+      const int total = warp_sum_i(nvalid);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)total * C::ROWB * 2);
+      __syncwarp();
+      if (nvalid > 0) {
+        const long long off = (long long)rb * (HKV * D);
+        if (nvalid == 4) {
+          bulk_g2s(kdst, a.k_pool + off, C::BLKB, &full[st]);
+          bulk_g2s(vdst, a.v_pool + off, C::BLKB, &full[st]);
+        } else {
+          for (int r = 0; r < nvalid; ++r) {
+            bulk_g2s(kdst + r * C::ROWB, a.k_pool + off + (long long)r * HKV * D, C::ROWB, &full[st]);
+            bulk_g2s(vdst + r * C::ROWB, a.v_pool + off + (long long)r * HKV * D, C::ROWB, &full[st]);
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ================================================================== consumers
+  const int g = warp % HKV;
+  const int slc = warp / HKV;
+  const int G = a.G;
+  const int qr = lane >> 2, qc = lane & 3;
+  // Q^T as the B operand: b0 = Q[head qr][16ks + 2qc ..], b1 = Q[head qr][16ks + 8 + 2qc ..]
+  uint32_t qb[D / 16][2];
+  {
+    const bool hv = ok && qr < G;
+    const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q + ((long long)row * a.Hq + g * G + qr) * D);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      qb[ks][0] = hv ? qp[ks * 8 + qc] : 0u;
+      qb[ks][1] = hv ? qp[ks * 8 + 4 + qc] : 0u;
+    }
+  }
+  float o[D / 16][4];  // O^T: rows = head dims (16 per m-tile), cols = heads
+#pragma unroll
+  for (int i = 0; i < D / 16; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2qc, 2qc+1
+  const float NEG = -INFINITY;
+  // this lane's ldmatrix row: MMA row ((lane&7) + 8*sel) -> slot (row&3), row-in-block (row>>2)
+  auto row_off = [&](int mrow) { return (4 * slc + (mrow & 3)) * C::BPITCH + (mrow >> 2) * C::ROWB; };
+  const int kr = (lane & 7) + (((lane >> 3) & 1) << 3);  // K: A-operand row of this lane
+  const int vr = (lane & 7) + ((lane >> 4) << 3);         // V^T: k (= position) row of this lane
+  const uint32_t koff = row_off(kr) + g * D * 2 + ((lane >> 4) << 4);
+  const uint32_t voff = row_off(vr) + g * D * 2 + (((lane >> 3) & 1) << 4);
+
+  for (int it = 0; it < nstages; ++it) {
+    const int st = it % C::NST;
+    if (!mbar_wait(&full[st], (it / C::NST) & 1, a.err)) break;
+    const int* pp = sPos + (st * C::NBS + 4 * slc) * 4;
+    const int pa = pp[(qr & 3) * 4 + (qr >> 2)];              // MMA row qr
+    const int pb = pp[((qr + 8) & 3) * 4 + ((qr + 8) >> 2)];  // MMA row qr + 8
+    if (__any_sync(0xffffffffu, pa >= 0 || pb >= 0)) {
+      const uint32_t kb = sbase + st * C::STAGE;
+      const uint32_t vb = kb + C::KVB;
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t kf[4];
+        ldsm_x4(kf, kb + koff + ks * 32);
+        mma_bf16_16816(s, kf, qb[ks][0], qb[ks][1]);
+      }
+      // s[0]=(row qr, head 2qc) s[1]=(qr, 2qc+1) s[2]=(qr+8, 2qc) s[3]=(qr+8, 2qc+1)
+      const float x0 = pa >= 0 ? s[0] * a.scale_log2 : NEG;
+      const float x1 = pa >= 0 ? s[1] * a.scale_log2 : NEG;
+      const float x2 = pb >= 0 ? s[2] * a.scale_log2 : NEG;
+      const float x3 = pb >= 0 ? s[3] * a.scale_log2 : NEG;
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int o2 = 4; o2 < 32; o2 <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = mn0 == NEG ? 1.f : exp2f(m0 - mn0);
+      const float al1 = mn1 == NEG ? 1.f : exp2f(m1 - mn1);
+      const float p0 = mn0 == NEG ? 0.f : exp2f(x0 - mn0);
+      const float p1 = mn1 == NEG ? 0.f : exp2f(x1 - mn1);
+      const float p2 = mn0 == NEG ? 0.f : exp2f(x2 - mn0);
+      const float p3 = mn1 == NEG ? 0.f : exp2f(x3 - mn1);
+      l0 = l0 * al0 + (p0 + p2);
+      l1 = l1 * al1 + (p1 + p3);
+      m0 = mn0;
+      m1 = mn1;
+#pragma unroll
+      for (int i = 0; i < D / 16; ++i) {
+        o[i][0] *= al0;
+        o[i][1] *= al1;
+        o[i][2] *= al0;
+        o[i][3] *= al1;
+      }
+      // P^T as the B operand (k = MMA row/position, n = head): transpose the two 8x8 blocks
+      const uint32_t pb0 = movmatrix_t(pack_bf16(p0, p1));
+      const uint32_t pb1 = movmatrix_t(pack_bf16(p2, p3));
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        uint32_t vf[4];
+        ldsm_x4_t(vf, vb + voff + mt * 32);
+        mma_bf16_16816(o[mt], vf, pb0, pb1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+
+  // ---- merge slices of each KV head through shared memory (consumer warps only)
+#pragma unroll
+  for (int o2 = 4; o2 < 32; o2 <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
+  }
+  asm volatile("bar.sync 1, %0;\n" ::"n"(C::NCW * 32));
+  float* sO = reinterpret_cast<float*>(smem) + warp * (8 * D + 16);  // [8 heads][D], m[8], l[8]
+  float* sM = sO + 8 * D;
+  float* sL = sM + 8;
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) {
+    const int d = mt * 16 + qr;
+    sO[(2 * qc) * D + d] = o[mt][0];
+    sO[(2 * qc + 1) * D + d] = o[mt][1];
+    sO[(2 * qc) * D + d + 8] = o[mt][2];
+    sO[(2 * qc + 1) * D + d + 8] = o[mt][3];
+  }
+  if (qr == 0) {
+    sM[2 * qc] = m0;
+    sM[2 * qc + 1] = m1;
+    sL[2 * qc] = l0;
+    sL[2 * qc + 1] = l1;
+  }
+  asm volatile("bar.sync 1, %0;\n" ::"n"(C::NCW * 32));
+  const int total = HKV * G * D;
+  for (int idx = tid; idx < total; idx += C::NCW * 32) {
+    const int gg = idx / (G * D);
+    const int h = (idx / D) % G;
+    const int d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int sl = 0; sl < C::NSLC; ++sl)
+      M = fmaxf(M, (reinterpret_cast<float*>(smem) + (sl * HKV + gg) * (8 * D + 16))[8 * D + h]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int sl = 0; sl < C::NSLC; ++sl) {
+        const float* base = reinterpret_cast<float*>(smem) + (sl * HKV + gg) * (8 * D + 16);
+        const float ms = base[8 * D + h];
+        if (ms != -INFINITY) {
+          const float f = exp2f(ms - M);
+          L += base[8 * D + 8 + h] * f;
+          O += base[h * D + d] * f;
+        }
+      }
+    }
+    const int hq = gg * G + h;
+    const float res = L > 0.f ? O / L : 0.f;
+    const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
+    if (a.splits == 1) {
+      a.out[((long long)row * a.Hq + hq) * D + d] = __float2bfloat16_rn(res);
+      if (a.lse && d == 0) a.lse[(long long)row * a.Hq + hq] = lse2 * 0.69314718055994531f;
+    } else {
+      const long long pi = ((long long)row * a.splits + split) * a.Hq + hq;
+      a.part_o[pi * D + d] = res;
+      if (d == 0) a.part_lse[pi] = lse2;
+    }
+  }
+}
+
 // Merge split-K partials: out = sum_s 2^(lse_s - L) o_s, L = log2 sum_s 2^lse_s.
 __global__ void combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                                int splits, int Hq, int D, bf16* __restrict__ out, float* lse) {
@@ -363,6 +664,14 @@ __global__ void combine_kernel(const float* __restrict__ part_o, const float* __
 
 template <int D, int HKV>
 cudaError_t run_sparse(const AttnArgs& a, int splits, cudaStream_t s) {
+  if (a.G <= 8) {
+    constexpr int SLC = kSwSlices<HKV>;
+    using C = SwCfg<D, HKV, SLC>;
+    cudaError_t e = set_smem_once(sparse_attn_sw_kernel<D, HKV, SLC>, C::TOTAL);
+    if (e != cudaSuccess) return e;
+    sparse_attn_sw_kernel<D, HKV, SLC><<<dim3(a.num_q, splits), C::THREADS, C::TOTAL, s>>>(a);
+    return cudaGetLastError();
+  }
   using C = AttnCfg<D, HKV>;
   cudaError_t e = set_smem_once(sparse_attn_kernel<D, HKV>, C::TOTAL);
   if (e != cudaSuccess) return e;

@@ -136,6 +136,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
+// L2 prefetch of a global range (no completion to track); bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------- ordering keys
 // Monotone map of fp32 onto uint32 (larger float -> larger integer); -0 is folded onto +0 by
 // the caller so that equal scores compare equal.

@@ -44,7 +44,7 @@ constexpr int TC_THREADS = (2 + TC_EPI) * 32;
 constexpr int TC_A_BYTES = 4 * 2 * TC_ROWS * 128;  // 4 heads x 2 K-halves x 128 rows x 128 B
 constexpr int TC_B_STAGE = 2 * TC_BLK * 128;       // 2 K-halves x 64 rows x 128 B
 constexpr int TC_B_BYTES = TC_NST * TC_B_STAGE;
-constexpr int TC_SCRATCH_KEYS = TC_B_BYTES / TC_EPI / 8;  // 1024 keys per epilogue warp
+constexpr int TC_SEL_MAX = TC_A_BYTES / TC_EPI / 8;  // 2048 keys per epilogue warp in the final select
 constexpr int TC_CAP = 2048;    // candidate slots per half-row
 
 struct TcMisc {
@@ -58,7 +58,6 @@ struct TcMisc {
   int cnt[2][TC_ROWS];
   float thr[2][TC_ROWS];
   float w[TC_ROWS][4];
-  uint32_t hist[TC_EPI][256];
 };
 constexpr int TC_SMEM = 1024 + TC_A_BYTES + TC_B_BYTES + (int)((sizeof(TcMisc) + 127) / 128 * 128);
 
@@ -171,7 +170,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 
   int it_base = 0;  // tiles of earlier segments (all roles count the same tiles)
-  bool first = true;
+  int segi = 0;     // segments started (phase of the query-tile barrier)
   for (;;) {
     __syncthreads();
     if (tid == 0) {
@@ -193,43 +192,61 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     if (warp == 0) {
       // ---------------------------------------------------------------- TMA producer
-      if (lane == 0) {
-        if (first) {
-          mbar_arrive_expect_tx(&m->aload, TC_A_BYTES);
-          for (int h = 0; h < 4; ++h)
-            for (int at = 0; at < 2; ++at)
-              tma3d(smem_addr(sA + (h * 2 + at) * (TC_ROWS * 128)), &tmA, at * 64, h, row0, &m->aload);
-        }
-        const int32_t* pt = a.page_table + (long long)seg * a.max_pages;
-        for (int i = 0; i < L; ++i) {
-          const int gi = it_base + i;
-          const int s = gi % TC_NST;
-          if (gi >= TC_NST && !mbar_wait(&m->empty[s], ((gi / TC_NST) & 1) ^ 1, a.err)) {
-            m->abort_flag = 1;
-            break;
-          }
-          const int tile = i < nsamp ? i * TC_SAMPLE : i - nsamp;
-          mbar_arrive_expect_tx(&m->full[s], TC_B_STAGE);
-          for (int pg = 0; pg < 4; ++pg) {
-            const int lp = tile * 4 + pg;
-            int page = 0;  // pages past the table hold only masked blocks; page 0 keeps the copy in bounds
-            if (lp < a.max_pages) {
+      // Page ids are fetched 8 tiles (32 pages) at a time, one per lane, so that no dependent
+      // page-table load sits between two tile issues; lane 0 issues the copies.
+      if (lane == 0) {  // query tiles, reloaded per segment (the final selection reuses sA)
+        mbar_arrive_expect_tx(&m->aload, TC_A_BYTES);
+        for (int h = 0; h < 4; ++h)
+          for (int at = 0; at < 2; ++at)
+            tma3d(smem_addr(sA + (h * 2 + at) * (TC_ROWS * 128)), &tmA, at * 64, h, row0, &m->aload);
+      }
+      const int32_t* pt = a.page_table + (long long)seg * a.max_pages;
+      bool stop = false;
+      for (int i0 = 0; i0 < L && !stop; i0 += 8) {
+        int mypage = 0;  // page of tile i0 + lane/4, page slot lane%4
+        {
+          const int i = i0 + (lane >> 2);
+          if (i < L) {
+            const int tile = i < nsamp ? i * TC_SAMPLE : i - nsamp;
+            const int lp = tile * 4 + (lane & 3);
+            if (lp < a.max_pages) {  // pages past the table hold only masked blocks: page 0
               const int p = pt[lp];
-              if (p >= 0 && p < a.num_pages) page = p;
+              if (p >= 0 && p < a.num_pages) mypage = p;
               else flag_error(a.err, QSA_DEVERR_PAGE);
             }
-            for (int at = 0; at < 2; ++at)
-              tma2d(smem_addr(sB + s * TC_B_STAGE + at * (TC_BLK * 128) + pg * 2048), &tmB, at * 64,
-                    page * 16, &m->full[s]);
           }
-          m->issued = gi + 1;
+        }
+        for (int j = 0; j < 8; ++j) {
+          const int i = i0 + j;
+          int pg4[4];
+#pragma unroll
+          for (int pg = 0; pg < 4; ++pg) pg4[pg] = __shfl_sync(0xffffffffu, mypage, j * 4 + pg);
+          if (i >= L) break;
+          if (lane == 0) {
+            const int gi = it_base + i;
+            const int s = gi % TC_NST;
+            if (gi >= TC_NST && !mbar_wait(&m->empty[s], ((gi / TC_NST) & 1) ^ 1, a.err)) {
+              m->abort_flag = 1;
+              stop = true;
+            } else {
+              mbar_arrive_expect_tx(&m->full[s], TC_B_STAGE);
+#pragma unroll
+              for (int pg = 0; pg < 4; ++pg)
+#pragma unroll
+                for (int at = 0; at < 2; ++at)
+                  tma2d(smem_addr(sB + s * TC_B_STAGE + at * (TC_BLK * 128) + pg * 2048), &tmB, at * 64,
+                        pg4[pg] * 16, &m->full[s]);
+              m->issued = gi + 1;
+            }
+          }
+          stop = __shfl_sync(0xffffffffu, stop, 0);
+          if (stop) break;
         }
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------------- MMA issuer
       if (lane == 0) {
-        bool ok = true;
-        if (first) ok = mbar_wait(&m->aload, 0, a.err);
+        bool ok = mbar_wait(&m->aload, segi & 1, a.err);
         for (int i = 0; ok && i < L; ++i) {
           const int gi = it_base + i;
           const int s = gi % TC_NST;
@@ -271,23 +288,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       u64* mybuf = cand + ((long long)(row0 + row) * 2 + hf) * TC_CAP;
       const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16);
       bool dead = false;
-      for (int i = 0; i < L; ++i) {
+      // -- sample tiles: keep the 32 best scores of this half-row in registers
+      for (int i = 0; i < nsamp && i < L; ++i) {
         const int gi = it_base + i;
         const int buf = gi & 1;
-        if (i == nsamp) {  // end of the sample: fix the row threshold (every epilogue warp arrives)
-          m->thr[hf][row] = (lim > a.topk) ? mn : -INFINITY;
-          epi_sync();
-          tau = fminf(m->thr[0][row], m->thr[1][row]);
-        }
-        if (dead) continue;
-        if (!mbar_wait(&m->tfull[buf], (gi >> 1) & 1, a.err)) {
+        if (!dead && !mbar_wait(&m->tfull[buf], (gi >> 1) & 1, a.err)) {
           m->abort_flag = 1;
           dead = true;
-          continue;
         }
+        if (dead) continue;
         tc_fence_after();
-        const bool sample = i < nsamp;
-        const int tile = sample ? i * TC_SAMPLE : i - nsamp;
+        const int tile = i * TC_SAMPLE;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           float v0[16], v1[16], v2[16], v3[16];
@@ -300,29 +311,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const int bbase = tile * TC_BLK + hf * 32 + c * 16;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            float s = w[0] * fmaxf(v0[j], 0.f);
-            s = fmaf(w[1], fmaxf(v1[j], 0.f), s);
-            s = fmaf(w[2], fmaxf(v2[j], 0.f), s);
-            s = fmaf(w[3], fmaxf(v3[j], 0.f), s);
-            const int b = bbase + j;
-            if (b < lim) {
-              if (sample) {
-                if (s > mn) {  // replace one current minimum, then recompute the minimum
-                  bool done = false;
+            float sc = w[0] * fmaxf(v0[j], 0.f);
+            sc = fmaf(w[1], fmaxf(v1[j], 0.f), sc);
+            sc = fmaf(w[2], fmaxf(v2[j], 0.f), sc);
+            sc = fmaf(w[3], fmaxf(v3[j], 0.f), sc);
+            if (bbase + j < lim && sc > mn) {  // replace one current minimum, recompute the min
+              bool done = false;
 #pragma unroll
-                  for (int k = 0; k < 32; ++k) {
-                    const bool hit = !done && top[k] == mn;
-                    top[k] = hit ? s : top[k];
-                    done |= hit;
-                  }
-                  mn = top[0];
-#pragma unroll
-                  for (int k = 1; k < 32; ++k) mn = fminf(mn, top[k]);
-                }
-              } else if (s >= tau) {
-                if (cnt < TC_CAP) mybuf[cnt] = make_key(s, (uint32_t)b);
-                ++cnt;
+              for (int k = 0; k < 32; ++k) {
+                const bool hit = !done && top[k] == mn;
+                top[k] = hit ? sc : top[k];
+                done |= hit;
               }
+              mn = top[0];
+#pragma unroll
+              for (int k = 1; k < 32; ++k) mn = fminf(mn, top[k]);
             }
           }
         }
@@ -330,76 +333,102 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&m->tempty[buf]);
       }
+      // -- row threshold: every epilogue warp arrives here once per segment with tiles
+      if (L > 0) {
+        m->thr[hf][row] = (lim > a.topk) ? mn : -INFINITY;
+        epi_sync();
+        tau = fminf(m->thr[0][row], m->thr[1][row]);
+      }
+      // -- all tiles: append every key with score >= tau (ascending block order per half-row)
+      for (int i = nsamp; i < L; ++i) {
+        const int gi = it_base + i;
+        const int buf = gi & 1;
+        if (!dead && !mbar_wait(&m->tfull[buf], (gi >> 1) & 1, a.err)) {
+          m->abort_flag = 1;
+          dead = true;
+        }
+        if (dead) continue;
+        tc_fence_after();
+        const int tile = i - nsamp;
+        float v[4][32];
+        const uint32_t col = tl + buf * 256 + hf * 32;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          tmem_ld16(col + h * TC_BLK, *reinterpret_cast<float(*)[16]>(&v[h][0]));
+          tmem_ld16(col + h * TC_BLK + 16, *reinterpret_cast<float(*)[16]>(&v[h][16]));
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&m->tempty[buf]);  // registers hold the tile: release TMEM early
+        const int bbase = tile * TC_BLK + hf * 32;
+        const bool full_tile = bbase + 32 <= lim;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float sc = w[0] * fmaxf(v[0][j], 0.f);
+          sc = fmaf(w[1], fmaxf(v[1][j], 0.f), sc);
+          sc = fmaf(w[2], fmaxf(v[2][j], 0.f), sc);
+          sc = fmaf(w[3], fmaxf(v[3][j], 0.f), sc);
+          const int b = bbase + j;
+          if (sc >= tau && (full_tile || b < lim)) {
+            if (cnt < TC_CAP) mybuf[cnt] = make_key(sc, (uint32_t)b);
+            ++cnt;
+          }
+        }
+      }
       m->cnt[hf][row] = cnt;
     }
     __syncthreads();  // the segment's tiles are all consumed; stage memory is free
 
     if (warp >= 2 && !m->abort_flag) {
       // ---------------------------------------------------------------- exact final selection
+      // Both half-row lists are ascending by block.  Find the need-th largest key of their union,
+      // keep the keys >= it from each list in order, and merge the two by rank.
       const int e = warp - 2;
-      u64* scratch = reinterpret_cast<u64*>(sB) + e * TC_SCRATCH_KEYS;
-      uint32_t* sblk = reinterpret_cast<uint32_t*>(scratch);
-      float* ssc = reinterpret_cast<float*>(sblk + 512);
+      u64* keys = reinterpret_cast<u64*>(sA) + e * TC_SEL_MAX;             // 16 KB per warp
+      uint32_t* hist = reinterpret_cast<uint32_t*>(sB) + e * 2048;         // 8 KB per warp
+      uint32_t* blk_a = hist;                                              // reused after the select
+      float* sc_a = reinterpret_cast<float*>(hist + 512);
+      uint32_t* blk_b = hist + 1024;
+      float* sc_b = reinterpret_cast<float*>(hist + 1536);
       for (int rr = 0; rr < 16; ++rr) {
         const int row = e * 16 + rr;
         if (m->seq[row] != seg) continue;
         const int lim = m->lim[row];
         const int need = min(a.topk, lim);
         const int n0 = m->cnt[0][row], n1 = m->cnt[1][row];
-        if (n0 > TC_CAP || n1 > TC_CAP || n0 + n1 < need) {
+        if (n0 > TC_CAP || n1 > TC_CAP || n0 + n1 < need || n0 + n1 > TC_SEL_MAX) {
           if (lane == 0) redo[row0 + row] = 1;
+          continue;
+        }
+        if (need == 0) {
+          write_selection(row0 + row, 0, lim, blk_a, sc_a, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
+          __syncwarp();
           continue;
         }
         const u64* rb = cand + (long long)(row0 + row) * 2 * TC_CAP;
         const int n = n0 + n1;
-        if (need > 0) {
-          u64* keys;
-          if (n <= TC_SCRATCH_KEYS) {
-            for (int i = lane; i < n; i += 32) scratch[i] = i < n0 ? rb[i] : rb[TC_CAP + i - n0];
-            keys = scratch;
-          } else {  // rare: pack both halves in place in global memory
-            u64* w = const_cast<u64*>(rb);
-            for (int base = 0; base < n1; base += 32) {
-              const int i = base + lane;
-              const u64 k = i < n1 ? w[TC_CAP + i] : 0ull;
-              __syncwarp();
-              if (i < n1) w[n0 + i] = k;
-              __syncwarp();
-            }
-            keys = w;
-          }
-          __syncwarp();
-          if (n > need) warp_select_compact(keys, n, need, m->hist[e]);
-          __syncwarp();
-          u64 kk[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) kk[u] = (lane + 32 * u) < need ? keys[lane + 32 * u] : 0ull;
-          __syncwarp();
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int i = lane + 32 * u;
-            if (i < need) {
-              sblk[i] = key_block(kk[u]);
-              ssc[i] = key_score(kk[u]);
-            }
-          }
-          __syncwarp();
-          warp_sort_blocks(sblk, ssc, need);
-        }
-        write_selection(row0 + row, need, lim, sblk, ssc, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
+        for (int i = lane; i < n; i += 32) keys[i] = i < n0 ? rb[i] : rb[TC_CAP + i - n0];
+        __syncwarp();
+        const u64 kth = warp_kth_largest(keys, n, need, hist);
+        __syncwarp();
+        const int na = warp_keep_sorted(keys, n0, kth, blk_a, sc_a);
+        const int nb2 = warp_keep_sorted(keys + n0, n1, kth, blk_b, sc_b);
+        warp_write_merged(row0 + row, blk_a, sc_a, na, blk_b, sc_b, nb2, lim, a.sel, a.n_sel,
+                          a.sel_scores, a.sel_stride);
         __syncwarp();
       }
     }
     __syncthreads();
     if (tid < TC_ROWS && m->seq[tid] == seg) m->seq[tid] = -1;
     it_base += L;
-    first = false;
+    ++segi;
   }
 
   // ---------------------------------------------------------------- teardown
   __syncthreads();
   if (m->abort_flag && warp == 0 && lane == 0) {  // let copies still in flight land first
-    mbar_wait(&m->aload, 0, a.err);
+    if (segi > 0) mbar_wait(&m->aload, (segi - 1) & 1, a.err);
     for (int gi = m->consumed; gi < m->issued; ++gi)
       mbar_wait(&m->full[gi % TC_NST], (gi / TC_NST) & 1, a.err);
   }

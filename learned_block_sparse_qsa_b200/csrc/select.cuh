@@ -10,14 +10,9 @@ namespace qsa {
 
 typedef unsigned long long u64;
 
-// Histogram increment with lanes that hit the same bin merged first (same-address shared-memory
-// atomics serialise).  Must be called by all 32 lanes of the warp.
+// Histogram increment (shared-memory atomic).  Called by all 32 lanes of the warp.
 __device__ __forceinline__ void hist_add(uint32_t* h, uint32_t bin, bool active) {
-  const unsigned am = __ballot_sync(0xffffffffu, active);
-  if (active) {
-    const unsigned peers = __match_any_sync(am, bin);
-    if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], (uint32_t)__popc(peers));
-  }
+  if (active) atomicAdd(&h[bin], 1u);
 }
 
 // One warp: find the `need`-th largest of the `cnt` unique keys in buf[0..cnt) by an MSB-first
@@ -119,6 +114,158 @@ __device__ __forceinline__ void warp_sort_blocks(uint32_t* blk, float* sc, int n
       __syncwarp();
     }
   }
+}
+
+// One warp: the need-th largest of n unique keys held in shared memory (keys[0..n)), 1 <= need <=
+// n.  MSB-first radix select with 11-bit digits that start at the highest bit where the keys
+// differ (found from their min and max), so the first pass already spreads them; histogram of
+// 2048 words in this warp's shared memory, plain shared atomics.
+__device__ __forceinline__ u64 warp_kth_largest(const u64* keys, int n, int need, uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  u64 lo = ~0ull, hi = 0ull;
+  for (int i = lane; i < n; i += 32) {
+    const u64 k = keys[i];
+    lo = k < lo ? k : lo;
+    hi = k > hi ? k : hi;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const u64 a = __shfl_xor_sync(0xffffffffu, lo, o), b = __shfl_xor_sync(0xffffffffu, hi, o);
+    lo = a < lo ? a : lo;
+    hi = b > hi ? b : hi;
+  }
+  if (need == n) return lo;
+  if (need == 1) return hi;
+  int top = 63 - __clzll((long long)(lo ^ hi));  // highest differing bit (lo != hi since n >= 2)
+  u64 prefix = hi & ~((2ull << top) - 1ull);     // bits above `top` are common to every key
+  u64 mask = ~((2ull << top) - 1ull);
+  if (top == 63) { prefix = 0; mask = 0; }
+  uint32_t remaining = (uint32_t)need;
+  for (;;) {
+    const int width = top + 1 < 11 ? top + 1 : 11;
+    const int shift = top + 1 - width;
+    const uint32_t nb = 1u << width;
+    for (uint32_t i = lane; i < nb; i += 32) hist[i] = 0;
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+      const u64 k = keys[i];
+      if ((k & mask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & (nb - 1)], 1u);
+    }
+    __syncwarp();
+    // lane l owns a contiguous run of bins counted from the top
+    const uint32_t per = (nb + 31) / 32;
+    uint32_t tot = 0;
+    for (uint32_t j = 0; j < per; ++j) {
+      const int bin = (int)nb - 1 - (int)(lane * per + j);
+      if (bin >= 0) tot += hist[bin];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - tot;
+    const bool mine = excl < remaining && remaining <= incl;
+    int digit = 0;
+    uint32_t above = 0, cnt_at = 0;
+    if (mine) {
+      uint32_t acc = excl;
+      for (uint32_t j = 0; j < per; ++j) {
+        const int bin = (int)nb - 1 - (int)(lane * per + j);
+        if (bin < 0) break;
+        const uint32_t c = hist[bin];
+        if (acc + c >= remaining) {
+          digit = bin;
+          above = acc;
+          cnt_at = c;
+          break;
+        }
+        acc += c;
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    cnt_at = __shfl_sync(0xffffffffu, cnt_at, src);
+    remaining -= above;
+    prefix |= (u64)digit << shift;
+    mask |= (u64)(nb - 1) << shift;
+    __syncwarp();
+    if (shift == 0) return prefix;  // every bit fixed: the key itself
+    if (cnt_at == remaining) {      // all keys under this prefix are kept: the answer is their min
+      u64 m = ~0ull;
+      for (int i = lane; i < n; i += 32) {
+        const u64 k = keys[i];
+        if ((k & mask) == prefix && k < m) m = k;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const u64 a = __shfl_xor_sync(0xffffffffu, m, o);
+        m = a < m ? a : m;
+      }
+      return m;
+    }
+    top = shift - 1;
+  }
+}
+
+// One warp: keep the keys >= kth of a list that is sorted by block, preserving that order;
+// writes blocks and scores to out_blk / out_sc and returns the count.
+__device__ __forceinline__ int warp_keep_sorted(const u64* keys, int n, u64 kth, uint32_t* out_blk,
+                                                float* out_sc) {
+  const int lane = threadIdx.x & 31;
+  int w = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const u64 k = i < n ? keys[i] : 0ull;
+    const bool keep = i < n && k >= kth;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int p = w + __popc(bal & ((1u << lane) - 1u));
+      out_blk[p] = key_block(k);
+      out_sc[p] = key_score(k);
+    }
+    w += __popc(bal);
+  }
+  __syncwarp();
+  return w;
+}
+
+// One warp: write the union of two ascending, disjoint block lists (a: na, b: nb) plus the tail
+// as one selection row, placing each element at its rank (own index + elements of the other
+// list with a smaller block, by binary search).
+__device__ __forceinline__ void warp_write_merged(int row, const uint32_t* ab, const float* as, int na,
+                                                  const uint32_t* bb, const float* bs, int nbk,
+                                                  int tail, int32_t* sel, int32_t* n_sel,
+                                                  float* sel_scores, int stride) {
+  const int lane = threadIdx.x & 31;
+  int32_t* srow = sel + (long long)row * stride;
+  float* crow = sel_scores ? sel_scores + (long long)row * stride : nullptr;
+  for (int side = 0; side < 2; ++side) {
+    const uint32_t* x = side ? bb : ab;
+    const float* xs = side ? bs : as;
+    const int nx = side ? nbk : na;
+    const uint32_t* y = side ? ab : bb;
+    const int ny = side ? na : nbk;
+    for (int i = lane; i < nx; i += 32) {
+      const uint32_t v = x[i];
+      int lo = 0, hi = ny;  // count of y < v
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (y[mid] < v) lo = mid + 1;
+        else hi = mid;
+      }
+      srow[i + lo] = (int32_t)v;
+      if (crow) crow[i + lo] = xs[i];
+    }
+  }
+  const int n = na + nbk;
+  for (int i = n + lane; i < stride; i += 32) {
+    srow[i] = i == n ? tail : -1;
+    if (crow) crow[i] = i == n ? __int_as_float(0x7f800000) : __int_as_float(0x7fc00000);
+  }
+  if (lane == 0) n_sel[row] = n + 1;
 }
 
 // Row whose query position or sequence failed validation: n_sel = 0, every entry -1.

@@ -91,3 +91,10 @@ def test_tc_fallback_on_decreasing_scores():
         check_selection(o["sel"][r], o["n_sel"][r], o["sel_scores"][r], ref_sel, ref_s, t, c.topk, True)
         if t // 4 > 512:
             assert list(ref_sel[:-1]) == list(range(512))  # the earliest blocks win
+
+
+def test_tc_decode_shaped_tile_with_four_sequences():
+    """4 sequences x 4 positions share one 128-row tile: four segments processed in turn."""
+    c = Config("tc_decode_b4x4", "decode", 4, 8192, 4, 8, 2, 64, 4, 128, shuffle_pages=True, seed=0x7C03)
+    run = Run(c, integer=True, score_path=1).step()
+    check_rows(run, range(c.num_q), True)
