@@ -156,7 +156,7 @@ def traffic_for(kernel_file: str, key: str):
 class Workload:
     """Device inputs + runner for one config (the prefix of the context already compressed)."""
 
-    def __init__(self, name: str, device):
+    def __init__(self, name: str, device, chunk: int = 0):
         import torch
 
         from learned_block_sparse_qsa_b200 import QsaConfig, QsaRunner
@@ -164,7 +164,7 @@ class Workload:
         from qsa_synth.device import DeviceInputs
 
         self.torch = torch
-        self.c = c = CONFIGS[name]
+        self.c = c = CONFIGS[name] if not chunk else CONFIGS[name].replace(n_new=chunk)
         self.di = d = DeviceInputs(c, integer=False, device=device)
         self.cfg = QsaConfig.make(c.Hq, c.Hkv, c.D, c.Di, topk=c.topk)
         self.runner = QsaRunner(self.cfg, device)
@@ -440,6 +440,8 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--case", default="", help="time one workload (C1..C5) only, per stage")
+    ap.add_argument("--chunk", type=int, default=0, help="with --case: new tokens per sequence")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -466,6 +468,15 @@ def main():
         return
 
     import torch
+
+    if args.case:  # one workload (e.g. a smaller chunk of the 1M-context prefill for ncu)
+        torch.cuda.set_device(local)
+        w = Workload(args.case, torch.device("cuda", local), args.chunk)
+        decode = w.c.mode == "decode"
+        stage_ms, step_ms, total_ms = time_steps(w, decode, args.steps, args.warmup, None)
+        print(json.dumps({"case": w.c.name, "num_q": w.c.num_q, "ms_per_step": total_ms / args.steps,
+                          "stages_ms": stage_ms}))
+        return
 
     dist = None
     if world > 1:
