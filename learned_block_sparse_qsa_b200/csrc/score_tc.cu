@@ -8,22 +8,25 @@
 // never be stored, so the selection is fused into the epilogue.
 //
 // CTA = 128 query rows (M = 128, one sequence segment at a time), warp-specialised:
-//   warp 0      TMA producer: the 4 heads' query tiles once (128 KB), then 64-block tiles of the
-//               compressed keys (4 pages x 2 K-halves of 16 rows x 128 B, 128-byte swizzle) into a
-//               4-stage ring;
-//   warp 1      owns the TMEM allocation (512 columns = two accumulator buffers x 4 heads x 64
-//               blocks) and one lane issues 4 x 8 tcgen05.mma (M=128, N=64, K=16) per tile;
+//   warp 0      TMA producer: the 4 heads' query tiles (128 KB), then 128-block tiles of the
+//               compressed keys (8 pages x 2 K-halves of 16 rows x 128 B, 128-byte swizzle) into a
+//               3-stage ring (96 KB);
+//   warp 1      owns the TMEM allocation (512 columns: pair X = heads 0,1 and pair Y = heads 2,3,
+//               each 2 x 128 blocks) and one lane issues 2 x 8 tcgen05.mma (M=128, N=128, K=16)
+//               into X, then 2 x 8 into Y, per tile; N=128 keeps the tensor pipe fed from shared
+//               memory (each MMA re-reads its 4 KB query slice for 2x the work of N=64);
 //   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (= its 32 query rows) and half of
-//               the 64 columns; thread = (query row, column half).
-// Selection without in-loop compaction: the tile sequence is first every 16th tile (a sample),
+//               the 128 columns; thread = (query row, column half).  The weighted ReLU sum of pair
+//               X stays in registers while pair Y is computed, then X and Y are released in turn.
+// Selection without in-loop compaction: the tile sequence is first every 32nd tile (a sample),
 // then all tiles.  During the sample each thread keeps the 32 best sampled scores of its half-row
-// in registers; the row threshold tau = min over its two halves of the 32nd best, so about 1,024
-// of the row's scores are >= tau.  The full pass appends every (score >= tau, block) key to a
-// per-half-row buffer; the final step checks that at least min(512, t/4) keys were kept -- which
-// proves every true top-512 key was kept -- and selects exactly (radix select on 64-bit keys,
-// lower block index wins ties).  Rows that fail the check (adversarial score orders) or overflow
-// the buffer are recomputed by the exact streaming kernel, so the result never depends on the
-// sample.
+// in registers; the row threshold tau = min over its two halves of the 32nd best, so about 2,048
+// of the row's scores are >= tau, and fewer than 512 is a ~6-sigma event.  The full pass appends every (score >= tau, block) key to a
+// per-half-row buffer (in ascending block order); the final step checks that at least
+// min(512, t/4) keys were kept -- which proves every true top-512 key was kept -- and selects
+// exactly (radix select on 64-bit keys, lower block index wins ties) with a merge by rank.  Rows
+// that fail the check (adversarial score orders) or overflow the buffer are recomputed by the exact
+// streaming kernel, so the result never depends on the sample.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -36,30 +39,33 @@ namespace qsa {
 namespace {
 
 constexpr int TC_ROWS = 128;
-constexpr int TC_BLK = 64;      // blocks per tile (MMA N)
-constexpr int TC_NST = 4;       // compressed-key stages
-constexpr int TC_SAMPLE = 16;   // every 16th tile is sampled
-constexpr int TC_EPI = 8;       // epilogue warps
+constexpr int TC_BLK = 128;           // blocks per tile (MMA N)
+constexpr int TC_PG = TC_BLK / 16;    // pages per tile
+constexpr int TC_NST = 3;             // compressed-key stages
+constexpr int TC_SAMPLE = 32;         // every 32nd tile is sampled
+constexpr int TC_EPI = 8;             // epilogue warps
 constexpr int TC_THREADS = (2 + TC_EPI) * 32;
 constexpr int TC_A_BYTES = 4 * 2 * TC_ROWS * 128;  // 4 heads x 2 K-halves x 128 rows x 128 B
-constexpr int TC_B_STAGE = 2 * TC_BLK * 128;       // 2 K-halves x 64 rows x 128 B
+constexpr int TC_B_STAGE = 2 * TC_BLK * 128;       // 2 K-halves x 128 rows x 128 B
 constexpr int TC_B_BYTES = TC_NST * TC_B_STAGE;
-constexpr int TC_SEL_MAX = TC_A_BYTES / TC_EPI / 8;  // 2048 keys per epilogue warp in the final select
-constexpr int TC_CAP = 2048;    // candidate slots per half-row
+constexpr int TC_CAP = 2048;          // candidate slots per half-row
 
 struct TcMisc {
+  // tfull/tempty[0]: TMEM pair X (heads 0, 1); [1]: pair Y (heads 2, 3)
   uint64_t full[TC_NST], empty[TC_NST], tfull[2], tempty[2], aload, mma_done;
   uint32_t tmem_base;
   int abort_flag;
   int issued, consumed;  // B tiles issued by the producer / waited for by the MMA issuer
   int seg, nb;
+  uint32_t done[4];      // rows already selected (bit per row)
+  uint32_t inseg[4];     // rows of the current segment
   int lim[TC_ROWS];
-  int seq[TC_ROWS];
   int cnt[2][TC_ROWS];
   float thr[2][TC_ROWS];
-  float w[TC_ROWS][4];
 };
-constexpr int TC_SMEM = 1024 + TC_A_BYTES + TC_B_BYTES + (int)((sizeof(TcMisc) + 127) / 128 * 128);
+// operands + bookkeeping; the dynamic shared-memory base must be 1024-byte aligned (checked)
+constexpr int TC_SMEM = TC_A_BYTES + TC_B_BYTES + (int)((sizeof(TcMisc) + 127) / 128 * 128);
+static_assert(TC_SMEM <= 232448, "shared memory budget");
 
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
   uint64_t d = (uint64_t)((addr >> 4) & 0x3FFF);
@@ -69,7 +75,7 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
   d |= (uint64_t)2 << 61;            // 128-byte swizzle
   return d;
 }
-// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M=128, N=64.
+// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M=128, N=128.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_BLK >> 3) << 17) |
                             ((uint32_t)(TC_ROWS >> 4) << 24);
 
@@ -113,18 +119,24 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
+__device__ __forceinline__ bool bit_of(const uint32_t* b, int i) { return (b[i >> 5] >> (i & 31)) & 1u; }
+
 __global__ void __launch_bounds__(TC_THREADS, 1)
     score_tc_kernel(ScoreArgs a, const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB, u64* __restrict__ cand,
                     int32_t* __restrict__ redo) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sA = smem;
   uint8_t* sB = smem + TC_A_BYTES;
   TcMisc* m = reinterpret_cast<TcMisc*>(sB + TC_B_BYTES);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row0 = blockIdx.x * TC_ROWS;
 
+  if (smem_addr(smem) & 1023) {  // operand tiles need 1024-byte alignment: leave the rows to the
+    if (tid < TC_ROWS && row0 + tid < a.num_q) redo[row0 + tid] = 1;  // exact streaming kernel
+    if (tid == 0) flag_error(a.err, QSA_DEVERR_INTERNAL);
+    return;
+  }
   if (tid == 0) {
     for (int s = 0; s < TC_NST; ++s) {
       mbar_init(&m->full[s], 1);
@@ -153,11 +165,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       lim = row_limit(a, r, &seq);
       redo[r] = 0;
     }
-    m->seq[tid] = lim >= 0 ? seq : -1;
     m->lim[tid] = lim;
-#pragma unroll
-    for (int h = 0; h < 4; ++h)
-      m->w[tid][h] = r < a.num_q ? __bfloat162float(a.idx_w[(long long)r * kHi + h]) : 0.f;
+    const unsigned bal = __ballot_sync(0xffffffffu, lim < 0);  // invalid rows count as done
+    if (lane == 0) m->done[tid >> 5] = bal;
   }
   tc_fence_before();
   __syncthreads();
@@ -173,15 +183,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   int segi = 0;     // segments started (phase of the query-tile barrier)
   for (;;) {
     __syncthreads();
-    if (tid == 0) {
-      int seg = -1, nb = 0;
-      for (int r = 0; r < TC_ROWS; ++r)
-        if (m->seq[r] >= 0) { seg = m->seq[r]; break; }
-      if (seg >= 0)
-        for (int r = 0; r < TC_ROWS; ++r)
-          if (m->seq[r] == seg) nb = max(nb, m->lim[r]);
-      m->seg = seg;
-      m->nb = nb;
+    if (warp == 0) {  // next segment: the sequence of the first row not yet done
+      int seg = -1;
+      for (int r = 0; r < TC_ROWS && seg < 0; ++r)
+        if (!bit_of(m->done, r)) seg = a.q_seq[row0 + r];
+      int nb = 0;
+      for (int r = lane; r < TC_ROWS; r += 32) {
+        const bool in = seg >= 0 && !bit_of(m->done, r) && a.q_seq[row0 + r] == seg;
+        const unsigned bal = __ballot_sync(0xffffffffu, in);
+        if (lane == 0) m->inseg[r >> 5] = bal;
+        if (in) nb = max(nb, m->lim[r]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) nb = max(nb, __shfl_xor_sync(0xffffffffu, nb, o));
+      if (lane == 0) {
+        m->seg = seg;
+        m->nb = nb;
+      }
     }
     __syncthreads();
     const int seg = m->seg;
@@ -192,7 +210,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     if (warp == 0) {
       // ---------------------------------------------------------------- TMA producer
-      // Page ids are fetched 8 tiles (32 pages) at a time, one per lane, so that no dependent
+      // Page ids are fetched several tiles at a time, one per lane, so that no dependent
       // page-table load sits between two tile issues; lane 0 issues the copies.
       if (lane == 0) {  // query tiles, reloaded per segment (the final selection reuses sA)
         mbar_arrive_expect_tx(&m->aload, TC_A_BYTES);
@@ -202,13 +220,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       const int32_t* pt = a.page_table + (long long)seg * a.max_pages;
       bool stop = false;
-      for (int i0 = 0; i0 < L && !stop; i0 += 8) {
-        int mypage = 0;  // page of tile i0 + lane/4, page slot lane%4
+      for (int i0 = 0; i0 < L && !stop; i0 += 32 / TC_PG) {
+        int mypage = 0;  // page slot lane%TC_PG of tile i0 + lane/TC_PG
         {
-          const int i = i0 + (lane >> 2);
+          const int i = i0 + lane / TC_PG;
           if (i < L) {
             const int tile = i < nsamp ? i * TC_SAMPLE : i - nsamp;
-            const int lp = tile * 4 + (lane & 3);
+            const int lp = tile * TC_PG + (lane % TC_PG);
             if (lp < a.max_pages) {  // pages past the table hold only masked blocks: page 0
               const int p = pt[lp];
               if (p >= 0 && p < a.num_pages) mypage = p;
@@ -216,11 +234,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
         }
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 32 / TC_PG; ++j) {
           const int i = i0 + j;
-          int pg4[4];
+          int pgs[TC_PG];
 #pragma unroll
-          for (int pg = 0; pg < 4; ++pg) pg4[pg] = __shfl_sync(0xffffffffu, mypage, j * 4 + pg);
+          for (int pg = 0; pg < TC_PG; ++pg) pgs[pg] = __shfl_sync(0xffffffffu, mypage, j * TC_PG + pg);
           if (i >= L) break;
           if (lane == 0) {
             const int gi = it_base + i;
@@ -231,11 +249,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             } else {
               mbar_arrive_expect_tx(&m->full[s], TC_B_STAGE);
 #pragma unroll
-              for (int pg = 0; pg < 4; ++pg)
+              for (int pg = 0; pg < TC_PG; ++pg)
 #pragma unroll
                 for (int at = 0; at < 2; ++at)
                   tma2d(smem_addr(sB + s * TC_B_STAGE + at * (TC_BLK * 128) + pg * 2048), &tmB, at * 64,
-                        pg4[pg] * 16, &m->full[s]);
+                        pgs[pg] * 16, &m->full[s]);
               m->issued = gi + 1;
             }
           }
@@ -250,24 +268,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int i = 0; ok && i < L; ++i) {
           const int gi = it_base + i;
           const int s = gi % TC_NST;
-          const int buf = gi & 1;
           if (!mbar_wait(&m->full[s], (gi / TC_NST) & 1, a.err)) { ok = false; break; }
           m->consumed = gi + 1;
-          if (gi >= 2 && !mbar_wait(&m->tempty[buf], ((gi >> 1) & 1) ^ 1, a.err)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t bst = smem_addr(sB + s * TC_B_STAGE);
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const uint32_t ast = smem_addr(sA + h * 2 * (TC_ROWS * 128));
+          for (int pair = 0; pair < 2; ++pair) {
+            // pair X (heads 0,1) -> columns 0..255, pair Y (heads 2,3) -> columns 256..511
+            if (gi >= 1 && !mbar_wait(&m->tempty[pair], (gi - 1) & 1, a.err)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-              const uint64_t ad = sw128_desc(ast + (ks >> 2) * (TC_ROWS * 128) + (ks & 3) * 32);
-              const uint64_t bd = sw128_desc(bst + (ks >> 2) * (TC_BLK * 128) + (ks & 3) * 32);
-              mma_f16(tbase + buf * 256 + h * TC_BLK, ad, bd, ks > 0 ? 1u : 0u);
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t ast = smem_addr(sA + (pair * 2 + hh) * 2 * (TC_ROWS * 128));
+#pragma unroll
+              for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t ad = sw128_desc(ast + (ks >> 2) * (TC_ROWS * 128) + (ks & 3) * 32);
+                const uint64_t bd = sw128_desc(bst + (ks >> 2) * (TC_BLK * 128) + (ks & 3) * 32);
+                mma_f16(tbase + pair * 256 + hh * TC_BLK, ad, bd, ks > 0 ? 1u : 0u);
+              }
             }
+            mma_commit(&m->tfull[pair]);
           }
+          if (!ok) break;
           mma_commit(&m->empty[s]);
-          mma_commit(&m->tfull[buf]);
         }
         if (!ok) m->abort_flag = 1;
       }
@@ -276,51 +298,76 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int q = warp & 3;
       const int hf = (warp - 2) >> 2;
       const int row = q * 32 + lane;
-      const int lim = (m->seq[row] == seg) ? m->lim[row] : -1;
+      const int lim = bit_of(m->inseg, row) ? m->lim[row] : -1;
       float w[4];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) w[h] = m->w[row][h];
+      for (int h = 0; h < 4; ++h)
+        w[h] = row0 + row < a.num_q ? __bfloat162float(a.idx_w[(long long)(row0 + row) * kHi + h]) : 0.f;
       float top[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) top[k] = -INFINITY;
       float mn = -INFINITY, tau = -INFINITY;
       int cnt = 0;
       u64* mybuf = cand + ((long long)(row0 + row) * 2 + hf) * TC_CAP;
-      const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16);
+      const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + hf * 64;
       bool dead = false;
-      // -- sample tiles: keep the 32 best scores of this half-row in registers
-      for (int i = 0; i < nsamp && i < L; ++i) {
-        const int gi = it_base + i;
-        const int buf = gi & 1;
-        if (!dead && !mbar_wait(&m->tfull[buf], (gi >> 1) & 1, a.err)) {
-          m->abort_flag = 1;
-          dead = true;
+      // Scores of this thread's 64 blocks of tile gi: pair X folded into sc[] and released, then
+      // pair Y added and released.
+      auto load_scores = [&](int gi, float (&sc)[64]) -> bool {
+        const uint32_t ph = gi & 1;
+#pragma unroll
+        for (int pair = 0; pair < 2; ++pair) {
+          if (!dead && !mbar_wait(&m->tfull[pair], ph, a.err)) {
+            m->abort_flag = 1;
+            dead = true;
+          }
+          if (dead) return false;
+          tc_fence_after();
+          const float wa = w[pair * 2], wb = w[pair * 2 + 1];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float va[16], vb[16];
+            const uint32_t col = tl + pair * 256 + c * 16;
+            tmem_ld16(col, va);
+            tmem_ld16(col + TC_BLK, vb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float x = fmaf(wb, fmaxf(vb[j], 0.f), wa * fmaxf(va[j], 0.f));
+              sc[c * 16 + j] = pair == 0 ? x : sc[c * 16 + j] + x;
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&m->tempty[pair]);
         }
-        if (dead) continue;
-        tc_fence_after();
-        const int tile = i * TC_SAMPLE;
+        return true;
+      };
+      // -- sample tiles: keep the 32 best scores of this half-row in registers.  The hot loop is
+      // branch-free (bit masks of blocks above the current minimum); the rare insertions run from
+      // one copy of the replacement code.
+      for (int i = 0; i < nsamp && i < L; ++i) {
+        float sc[64];
+        if (!load_scores(it_base + i, sc)) continue;
+        const int bbase = i * TC_SAMPLE * TC_BLK + hf * 64;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float v0[16], v1[16], v2[16], v3[16];
-          const uint32_t col = tl + buf * 256 + hf * 32 + c * 16;
-          tmem_ld16(col + 0 * TC_BLK, v0);
-          tmem_ld16(col + 1 * TC_BLK, v1);
-          tmem_ld16(col + 2 * TC_BLK, v2);
-          tmem_ld16(col + 3 * TC_BLK, v3);
-          tmem_wait_ld();
-          const int bbase = tile * TC_BLK + hf * 32 + c * 16;
+        for (int half = 0; half < 2; ++half) {
+          uint32_t hits = 0;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float sc = w[0] * fmaxf(v0[j], 0.f);
-            sc = fmaf(w[1], fmaxf(v1[j], 0.f), sc);
-            sc = fmaf(w[2], fmaxf(v2[j], 0.f), sc);
-            sc = fmaf(w[3], fmaxf(v3[j], 0.f), sc);
-            if (bbase + j < lim && sc > mn) {  // replace one current minimum, recompute the min
+          for (int j = 0; j < 32; ++j)
+            hits |= (uint32_t)(sc[half * 32 + j] > mn && bbase + half * 32 + j < lim) << j;
+          while (hits) {
+            const int j = __ffs(hits) - 1;
+            hits &= hits - 1;
+            float x = sc[half * 32];
+#pragma unroll
+            for (int k = 1; k < 32; ++k) x = (j == k) ? sc[half * 32 + k] : x;
+            if (x > mn) {  // replace one current minimum, then recompute the minimum
               bool done = false;
 #pragma unroll
               for (int k = 0; k < 32; ++k) {
                 const bool hit = !done && top[k] == mn;
-                top[k] = hit ? sc : top[k];
+                top[k] = hit ? x : top[k];
                 done |= hit;
               }
               mn = top[0];
@@ -329,9 +376,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&m->tempty[buf]);
       }
       // -- row threshold: every epilogue warp arrives here once per segment with tiles
       if (L > 0) {
@@ -341,37 +385,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       // -- all tiles: append every key with score >= tau (ascending block order per half-row)
       for (int i = nsamp; i < L; ++i) {
-        const int gi = it_base + i;
-        const int buf = gi & 1;
-        if (!dead && !mbar_wait(&m->tfull[buf], (gi >> 1) & 1, a.err)) {
-          m->abort_flag = 1;
-          dead = true;
-        }
-        if (dead) continue;
-        tc_fence_after();
-        const int tile = i - nsamp;
-        float v[4][32];
-        const uint32_t col = tl + buf * 256 + hf * 32;
+        float sc[64];
+        if (!load_scores(it_base + i, sc)) continue;
+        const int bbase = (i - nsamp) * TC_BLK + hf * 64;
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          tmem_ld16(col + h * TC_BLK, *reinterpret_cast<float(*)[16]>(&v[h][0]));
-          tmem_ld16(col + h * TC_BLK + 16, *reinterpret_cast<float(*)[16]>(&v[h][16]));
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&m->tempty[buf]);  // registers hold the tile: release TMEM early
-        const int bbase = tile * TC_BLK + hf * 32;
-        const bool full_tile = bbase + 32 <= lim;
+        for (int half = 0; half < 2; ++half) {
+          const int nvalid = min(32, lim - bbase - half * 32);  // blocks below the causal limit
+          uint32_t hits = 0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float sc = w[0] * fmaxf(v[0][j], 0.f);
-          sc = fmaf(w[1], fmaxf(v[1][j], 0.f), sc);
-          sc = fmaf(w[2], fmaxf(v[2][j], 0.f), sc);
-          sc = fmaf(w[3], fmaxf(v[3][j], 0.f), sc);
-          const int b = bbase + j;
-          if (sc >= tau && (full_tile || b < lim)) {
-            if (cnt < TC_CAP) mybuf[cnt] = make_key(sc, (uint32_t)b);
+          for (int j = 0; j < 32; ++j) hits |= (uint32_t)(sc[half * 32 + j] >= tau) << j;
+          hits &= nvalid >= 32 ? 0xffffffffu : (nvalid <= 0 ? 0u : ((1u << nvalid) - 1u));
+          while (hits) {  // ascending block order
+            const int j = __ffs(hits) - 1;
+            hits &= hits - 1;
+            float x = sc[half * 32];
+#pragma unroll
+            for (int k = 1; k < 32; ++k) x = (j == k) ? sc[half * 32 + k] : x;
+            if (cnt < TC_CAP) mybuf[cnt] = make_key(x, (uint32_t)(bbase + half * 32 + j));
             ++cnt;
           }
         }
@@ -385,19 +415,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // Both half-row lists are ascending by block.  Find the need-th largest key of their union,
       // keep the keys >= it from each list in order, and merge the two by rank.
       const int e = warp - 2;
-      u64* keys = reinterpret_cast<u64*>(sA) + e * TC_SEL_MAX;             // 16 KB per warp
-      uint32_t* hist = reinterpret_cast<uint32_t*>(sB) + e * 2048;         // 8 KB per warp
-      uint32_t* blk_a = hist;                                              // reused after the select
+      uint32_t* hist = reinterpret_cast<uint32_t*>(sB) + e * 2048;  // 8 KB per warp
+      uint32_t* blk_a = hist;                                       // reused after the select
       float* sc_a = reinterpret_cast<float*>(hist + 512);
       uint32_t* blk_b = hist + 1024;
       float* sc_b = reinterpret_cast<float*>(hist + 1536);
       for (int rr = 0; rr < 16; ++rr) {
         const int row = e * 16 + rr;
-        if (m->seq[row] != seg) continue;
+        if (!bit_of(m->inseg, row)) continue;
         const int lim = m->lim[row];
         const int need = min(a.topk, lim);
         const int n0 = m->cnt[0][row], n1 = m->cnt[1][row];
-        if (n0 > TC_CAP || n1 > TC_CAP || n0 + n1 < need || n0 + n1 > TC_SEL_MAX) {
+        if (n0 > TC_CAP || n1 > TC_CAP || n0 + n1 < need) {
           if (lane == 0) redo[row0 + row] = 1;
           continue;
         }
@@ -406,21 +435,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           __syncwarp();
           continue;
         }
-        const u64* rb = cand + (long long)(row0 + row) * 2 * TC_CAP;
-        const int n = n0 + n1;
-        for (int i = lane; i < n; i += 32) keys[i] = i < n0 ? rb[i] : rb[TC_CAP + i - n0];
+        // the candidate buffers (L2-resident) are read in place
+        const u64* ka = cand + (long long)(row0 + row) * 2 * TC_CAP;
+        const u64* kb = ka + TC_CAP;
+        const u64 kth = warp_kth_largest2(ka, n0, kb, n0 + n1, need, hist);
         __syncwarp();
-        const u64 kth = warp_kth_largest(keys, n, need, hist);
-        __syncwarp();
-        const int na = warp_keep_sorted(keys, n0, kth, blk_a, sc_a);
-        const int nb2 = warp_keep_sorted(keys + n0, n1, kth, blk_b, sc_b);
+        const int na = warp_keep_sorted(ka, n0, kth, blk_a, sc_a);
+        const int nb2 = warp_keep_sorted(kb, n1, kth, blk_b, sc_b);
         warp_write_merged(row0 + row, blk_a, sc_a, na, blk_b, sc_b, nb2, lim, a.sel, a.n_sel,
                           a.sel_scores, a.sel_stride);
         __syncwarp();
       }
     }
     __syncthreads();
-    if (tid < TC_ROWS && m->seq[tid] == seg) m->seq[tid] = -1;
+    if (tid < 4) m->done[tid] |= m->inseg[tid];
     it_base += L;
     ++segi;
   }

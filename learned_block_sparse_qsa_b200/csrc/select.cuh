@@ -116,15 +116,24 @@ __device__ __forceinline__ void warp_sort_blocks(uint32_t* blk, float* sc, int n
   }
 }
 
-// One warp: the need-th largest of n unique keys held in shared memory (keys[0..n)), 1 <= need <=
+// One warp: the need-th largest of n unique keys (keys[0..n), shared or global memory), 1 <= need <=
 // n.  MSB-first radix select with 11-bit digits that start at the highest bit where the keys
 // differ (found from their min and max), so the first pass already spreads them; histogram of
 // 2048 words in this warp's shared memory, plain shared atomics.
+__device__ __forceinline__ u64 warp_kth_largest2(const u64* ka, int na, const u64* kb, int n, int need,
+                                                 uint32_t* hist);
 __device__ __forceinline__ u64 warp_kth_largest(const u64* keys, int n, int need, uint32_t* hist) {
+  return warp_kth_largest2(keys, n, nullptr, n, need, hist);
+}
+
+// Same over the concatenation of two arrays: ka[0..na) then kb[0..n-na).
+__device__ __forceinline__ u64 warp_kth_largest2(const u64* ka, int na, const u64* kb, int n, int need,
+                                                 uint32_t* hist) {
   const int lane = threadIdx.x & 31;
+  auto key_at = [&](int i) { return i < na ? ka[i] : kb[i - na]; };
   u64 lo = ~0ull, hi = 0ull;
   for (int i = lane; i < n; i += 32) {
-    const u64 k = keys[i];
+    const u64 k = key_at(i);
     lo = k < lo ? k : lo;
     hi = k > hi ? k : hi;
   }
@@ -148,7 +157,7 @@ __device__ __forceinline__ u64 warp_kth_largest(const u64* keys, int n, int need
     for (uint32_t i = lane; i < nb; i += 32) hist[i] = 0;
     __syncwarp();
     for (int i = lane; i < n; i += 32) {
-      const u64 k = keys[i];
+      const u64 k = key_at(i);
       if ((k & mask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & (nb - 1)], 1u);
     }
     __syncwarp();
@@ -196,7 +205,7 @@ __device__ __forceinline__ u64 warp_kth_largest(const u64* keys, int n, int need
     if (cnt_at == remaining) {      // all keys under this prefix are kept: the answer is their min
       u64 m = ~0ull;
       for (int i = lane; i < n; i += 32) {
-        const u64 k = keys[i];
+        const u64 k = key_at(i);
         if ((k & mask) == prefix && k < m) m = k;
       }
 #pragma unroll
