@@ -1,8 +1,8 @@
 """Build libqsa.so (this package) and libqsa_synth.so (the input generator) for sm_100a.
 
 Each .cu file is compiled to an object under _build/ in parallel, then linked with nvcc into a
-shared library placed next to its Python package.  Run ``python -m
-learned_block_sparse_qsa_b200.build`` (or ``__graft_entry__.build()``).
+shared library placed next to its Python package.  Run ``python learned_block_sparse_qsa_b200/build.py``
+(or ``__graft_entry__.build()``); it does not import the package, which needs the library.
 """
 from __future__ import annotations
 

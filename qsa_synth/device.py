@@ -15,7 +15,7 @@ from . import (TID_IDXK, TID_IDXQ, TID_IDXW, TID_K, TID_Q, TID_V, Config, HostIn
 
 _LIB = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqsa_synth.so")
 if not os.path.exists(_LIB):
-    raise ImportError(f"{_LIB} is missing: run `python -m learned_block_sparse_qsa_b200.build`")
+    raise ImportError(f"{_LIB} is missing: run `python learned_block_sparse_qsa_b200/build.py`")
 _lib = ctypes.CDLL(_LIB)
 _lib.qsyn_fill_linear.restype = ctypes.c_int
 _lib.qsyn_fill_linear.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_uint64,
