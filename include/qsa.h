@@ -157,6 +157,21 @@ qsa_status_t qsa_sparse_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* 
                                     float* lse, int32_t num_splits, void* workspace,
                                     size_t ws_bytes, qsa_stream_t stream);
 
+/* No counterpart in the article: a variant of qsa_sparse_attn_decode for callers that cannot
+ * allocate device memory at step time (for example a serving engine whose memory planner owns all
+ * device memory and forbids allocations after start-up, or a plug-in host that gives plug-ins no
+ * allocator).  Same arguments and results minus the workspace: the split-K partials live in a
+ * 4 MiB array of device memory owned by libqsa (held by every GPU that loads the library until
+ * the process exits).  num_splits > 0 whose partials (num_q * num_splits * Hq * (D + 1) floats)
+ * exceed 4 MiB is rejected with QSA_ERR_WORKSPACE; num_splits = 0 picks the automatic split count,
+ * lowered until the partials fit.  The first call on a device looks up the array's address (a
+ * synchronous runtime call) and should come before any stream capture.  All calls share the
+ * array: calls that overlap on the GPU race.  Nothing is allocated or freed. */
+qsa_status_t qsa_sparse_attn_decode_noalloc(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                            const void* q, const void* k_pool, const void* v_pool,
+                                            const int32_t* sel, const int32_t* n_sel, void* out,
+                                            float* lse, int32_t num_splits, qsa_stream_t stream);
+
 /* The comparison baseline (section "Three speed claims, three different experiments": paged
  * grouped-query attention): row i attends over every position 0..t of its sequence on the same
  * pools.  Rows of one sequence should be contiguous (they share key/value tiles).  Prefill form:

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libqsa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m learned_block_sparse_qsa_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python learned_block_sparse_qsa_b200/build.py` "
         "(nvcc, sm_100a). libqsa has no CPU fallback.")
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -84,6 +84,8 @@ _SIGS = {
                                           c_void_p, c_void_p, c_void_p]),
     "qsa_sparse_attn_decode": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
+    "qsa_sparse_attn_decode_noalloc": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                  c_void_p, c_void_p, c_void_p, c_int32, c_void_p]),
     "qsa_dense_attn_prefill": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_void_p]),
     "qsa_dense_attn_decode": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -148,6 +150,15 @@ def qsa_sparse_attn_decode(cfg, batch, q, k_pool, v_pool, sel, n_sel, out, lse, 
                                        _p(v_pool), _p(sel), _p(n_sel), _p(out), _p(lse),
                                        int(num_splits), _p(workspace), int(ws_bytes), _stream(stream)),
            "qsa_sparse_attn_decode")
+
+
+def qsa_sparse_attn_decode_noalloc(cfg, batch, q, k_pool, v_pool, sel, n_sel, out, lse=None,
+                                   num_splits=0, stream=None):
+    """Split-K decode attention with library-owned scratch (no workspace argument)."""
+    _check(_lib.qsa_sparse_attn_decode_noalloc(ctypes.byref(cfg), ctypes.byref(batch), _p(q),
+                                               _p(k_pool), _p(v_pool), _p(sel), _p(n_sel), _p(out),
+                                               _p(lse), int(num_splits), _stream(stream)),
+           "qsa_sparse_attn_decode_noalloc")
 
 
 def qsa_dense_attn_prefill(cfg, batch, q, k_pool, v_pool, out, lse=None, stream=None):
