@@ -491,7 +491,13 @@ def main():
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     gpu_index = int(vis.split(",")[local]) if vis and vis.split(",")[local].isdigit() else local
     l2_flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    flush = lambda: l2_flush_buf.zero_()  # noqa: E731
+    l2_flush_sum = torch.empty((), dtype=torch.int64, device=dev)
+
+    def flush():
+        # write a buffer twice the L2 size, then read it back: the timed step starts with an L2
+        # that holds none of its data and no dirty lines to write back
+        l2_flush_buf.zero_()
+        torch.sum(l2_flush_buf.view(torch.int64), dim=0, out=l2_flush_sum)
 
     # ---------------------------------------------------------------- prefill (headline)
     w = Workload(PREFILL, dev)
@@ -580,7 +586,7 @@ def main():
                        "q_heads": c.Hq, "kv_heads": c.Hkv, "head_dim": c.D, "idx_heads": c.Hi,
                        "idx_dim": c.Di, "topk_blocks": c.topk, "page_tokens": c.page,
                        "l2": "inputs larger than L2 (2 GiB paged KV gathered per step); decode "
-                             "steps flush L2 (256 MiB write) between timed steps",
+                             "steps flush L2 (256 MiB write + read back) between timed steps",
                        "parallelism": f"replicas x{world}"},
             "roofline": roofline,
             "stages_ms": {k: v["ms"] for k, v in stages.items()},

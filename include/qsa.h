@@ -38,6 +38,8 @@
  *   idx_q      bf16 [num_q, 4, Di]            indexer queries;  idx_w bf16 [num_q, 4] head weights
  *   sel        int32 [num_q, topk+1]          selected blocks, ascending, tail block last, -1 pad
  *   n_sel      int32 [num_q]                  min(topk, t/4) + 1
+ * q, k_pool, v_pool, kcomp_pool, idx_q, idx_k and the attention output must be 16-byte aligned
+ * (QSA_ERR_INVALID_ARG otherwise).
  */
 #ifndef QSA_H
 #define QSA_H
@@ -82,7 +84,8 @@ typedef struct qsa_config {
   int32_t topk_blocks;  /* 1..512; the article's budget is 512 */
   int32_t page_tokens;  /* must be 64 */
   float softmax_scale;  /* <= 0 selects 1/sqrt(head_dim) */
-  int32_t score_path;   /* qsa_index_score_topk algorithm: 0 auto, 1 streaming, 2 materialised */
+  int32_t score_path;   /* qsa_index_score_topk algorithm: 0 auto, 1 streaming, 2 materialised,
+                           3 split lists (idx_dim 128; falls back to 2 otherwise) */
 } qsa_config_t;
 
 typedef struct qsa_batch {
@@ -149,8 +152,9 @@ qsa_status_t qsa_sparse_attn_prefill(const qsa_config_t* cfg, const qsa_batch_t*
 /* Same result as qsa_sparse_attn_prefill, computed split-K for few query rows (decode with
  * multi-token prediction, section "Three speed claims, three different experiments"): each row's
  * selected blocks are cut into num_splits pieces (0 = chosen from the device) processed in
- * parallel, then merged by their log-sum-exp.  workspace: qsa_workspace_size(...,
- * QSA_OP_SPARSE_ATTN_DECODE, num_splits, ...) bytes. */
+ * parallel, then merged by their log-sum-exp (by the last piece of each row to finish, when
+ * Hq/Hkv <= 8; else by a second kernel).  workspace: qsa_workspace_size(...,
+ * QSA_OP_SPARSE_ATTN_DECODE, num_splits, ...) bytes; its contents need no initialisation. */
 qsa_status_t qsa_sparse_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* batch,
                                     const void* q, const void* k_pool, const void* v_pool,
                                     const int32_t* sel, const int32_t* n_sel, void* out,

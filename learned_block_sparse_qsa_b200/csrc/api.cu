@@ -49,7 +49,7 @@ qsa_status_t make_geometry(const qsa_config_t* cfg, const qsa_batch_t* b, Geomet
     return QSA_ERR_INVALID_ARG;
   if (!pow2_le(cfg->num_q_heads / cfg->num_kv_heads, 16)) return QSA_ERR_UNSUPPORTED;
   if (cfg->topk_blocks < 1 || cfg->topk_blocks > 512) return QSA_ERR_UNSUPPORTED;
-  if (cfg->score_path < 0 || cfg->score_path > 2) return QSA_ERR_INVALID_ARG;
+  if (cfg->score_path < 0 || cfg->score_path > 3) return QSA_ERR_INVALID_ARG;
   if ((long long)b->max_pages_per_seq * 64 > (1LL << 30)) return QSA_ERR_UNSUPPORTED;
   g->Hq = cfg->num_q_heads;
   g->Hkv = cfg->num_kv_heads;
@@ -100,11 +100,9 @@ qsa_status_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_batch_t* batc
     case QSA_OP_INDEX_SCORE_TOPK:
       *bytes = qsa::score_workspace_bytes(g, qsa::resolve_score_path(g, cfg->score_path));
       return QSA_OK;
-    case QSA_OP_SPARSE_ATTN_DECODE: {
-      const int s = qsa::resolve_sparse_splits(g, num_splits);
-      *bytes = s > 1 ? qsa::sparse_decode_workspace_bytes(g, s) : 0;
+    case QSA_OP_SPARSE_ATTN_DECODE:
+      *bytes = qsa::sparse_decode_workspace_bytes(g, qsa::resolve_sparse_splits(g, num_splits));
       return QSA_OK;
-    }
     case QSA_OP_DENSE_ATTN_DECODE: {
       const int s = qsa::resolve_dense_splits(g, num_splits);
       *bytes = s > 1 ? qsa::dense_decode_workspace_bytes(g, s) : 0;
@@ -173,7 +171,7 @@ static qsa_status_t sparse_common(const qsa_config_t* cfg, const qsa_batch_t* ba
   if (g->num_q == 0) return QSA_OK;
   if (!q || !k_pool || !v_pool || !sel || !n_sel || !out) return QSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k_pool) |
-       reinterpret_cast<uintptr_t>(v_pool)) & 15)
+       reinterpret_cast<uintptr_t>(v_pool) | reinterpret_cast<uintptr_t>(out)) & 15)
     return QSA_ERR_INVALID_ARG;
   return QSA_OK;
 }
@@ -199,11 +197,9 @@ qsa_status_t qsa_sparse_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* 
   if (st != QSA_OK || g.num_q == 0) return st;
   if (num_splits < 0) return QSA_ERR_INVALID_ARG;
   const int s = qsa::resolve_sparse_splits(g, num_splits);
-  if (s > 1) {
-    const size_t need = qsa::sparse_decode_workspace_bytes(g, s);
-    if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
-      return QSA_ERR_WORKSPACE;
-  }
+  const size_t need = qsa::sparse_decode_workspace_bytes(g, s);
+  if (need > 0 && (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)))
+    return QSA_ERR_WORKSPACE;
   return from_cuda(qsa::launch_sparse_attn(g, q, k_pool, v_pool, sel, n_sel, g.topk + 1, out,
                                            lse, s, workspace, (cudaStream_t)stream));
 }

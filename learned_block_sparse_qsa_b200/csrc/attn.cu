@@ -41,8 +41,10 @@ struct AttnArgs {
   float* part_o;
   float* part_lse;
   int splits;
+  uint32_t* arrivals;  // split-K: per-row count of finished splits (zeroed before the launch)
   int32_t* err;
 };
+
 
 template <int D, int HKV>
 struct AttnCfg {
@@ -415,13 +417,10 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
     }
     mbar_fence_init();
   }
-  __syncthreads();
-
-  if (warp == C::NCW) {
-    // ================================================================ producer
+  {  // every thread: one round of (selection entry -> page table) loads for the CTA's slice
     const int32_t* selrow = a.sel + (long long)row * a.sel_stride;
     const int32_t* ptab = a.page_table + (long long)(ok ? seq : 0) * a.max_pages;
-    for (int i = lane; i < nblk; i += 32) {  // selection slice -> physical row bases
+    for (int i = tid; i < nblk; i += C::THREADS) {
       const int b = selrow[blo + i];
       int rb = -1;
       if (b < 0 || b > t / 4) {
@@ -434,7 +433,11 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
       sRow[i] = rb;
       sBlk[i] = b;
     }
-    __syncwarp();
+  }
+  __syncthreads();
+
+  if (warp == C::NCW) {
+    // ================================================================ producer
     for (int it = 0; it < nstages; ++it) {
       const int st = it % C::NST;
       if (it >= C::NST && !mbar_wait(&empty[st], ((it / C::NST) - 1) & 1, a.err)) break;
@@ -483,9 +486,7 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
         }
       }
     }
-    return;
-  }
-
+  } else {
   // ================================================================== consumers
   const int g = warp % HKV;
   const int slc = warp / HKV;
@@ -600,38 +601,100 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
     sL[2 * qc + 1] = l1;
   }
   asm volatile("bar.sync 1, %0;\n" ::"n"(C::NCW * 32));
-  const int total = HKV * G * D;
-  for (int idx = tid; idx < total; idx += C::NCW * 32) {
-    const int gg = idx / (G * D);
-    const int h = (idx / D) % G;
-    const int d = idx % D;
-    float M = -INFINITY;
+  // one warp per (KV head gg, query head h of its group), lanes across the head dims
+  const int lg = __ffs(G) - 1;  // G is a power of two
+  for (int c = warp; c < HKV * G; c += C::NCW) {
+    const int gg = c >> lg, h = c & (G - 1);
+    float f[C::NSLC];
+    float M = -INFINITY, L = 0.f;
 #pragma unroll
     for (int sl = 0; sl < C::NSLC; ++sl)
       M = fmaxf(M, (reinterpret_cast<float*>(smem) + (sl * HKV + gg) * (8 * D + 16))[8 * D + h]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
 #pragma unroll
-      for (int sl = 0; sl < C::NSLC; ++sl) {
-        const float* base = reinterpret_cast<float*>(smem) + (sl * HKV + gg) * (8 * D + 16);
-        const float ms = base[8 * D + h];
-        if (ms != -INFINITY) {
-          const float f = exp2f(ms - M);
-          L += base[8 * D + 8 + h] * f;
-          O += base[h * D + d] * f;
-        }
-      }
+    for (int sl = 0; sl < C::NSLC; ++sl) {
+      const float* base = reinterpret_cast<float*>(smem) + (sl * HKV + gg) * (8 * D + 16);
+      const float ms = base[8 * D + h];
+      f[sl] = (M != -INFINITY && ms != -INFINITY) ? exp2f(ms - M) : 0.f;
+      L += base[8 * D + 8 + h] * f[sl];
     }
     const int hq = gg * G + h;
-    const float res = L > 0.f ? O / L : 0.f;
+    const float inv = L > 0.f ? 1.0f / L : 0.f;
     const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
-    if (a.splits == 1) {
-      a.out[((long long)row * a.Hq + hq) * D + d] = __float2bfloat16_rn(res);
-      if (a.lse && d == 0) a.lse[(long long)row * a.Hq + hq] = lse2 * 0.69314718055994531f;
-    } else {
-      const long long pi = ((long long)row * a.splits + split) * a.Hq + hq;
-      a.part_o[pi * D + d] = res;
-      if (d == 0) a.part_lse[pi] = lse2;
+    const long long pi = ((long long)row * a.splits + split) * a.Hq + hq;
+    for (int d = lane; d < D; d += 32) {
+      float O = 0.f;
+#pragma unroll
+      for (int sl = 0; sl < C::NSLC; ++sl)
+        O += (reinterpret_cast<float*>(smem) + (sl * HKV + gg) * (8 * D + 16))[h * D + d] * f[sl];
+      const float res = O * inv;
+      if (a.splits == 1) a.out[((long long)row * a.Hq + hq) * D + d] = __float2bfloat16_rn(res);
+      else a.part_o[pi * D + d] = res;
+    }
+    if (lane == 0) {
+      if (a.splits == 1) {
+        if (a.lse) a.lse[(long long)row * a.Hq + hq] = lse2 * 0.69314718055994531f;
+      } else {
+        a.part_lse[pi] = lse2;
+      }
+    }
+  }
+  }  // consumers
+
+  if (a.splits > 1) {
+    // the last split of the row to finish merges all of the row's partials (log-sum-exp weights)
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&a.arrivals[row], 1u) == (uint32_t)a.splits - 1u;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      const int S = a.splits, Hq = a.Hq;
+      const long long b0 = (long long)row * S * Hq;  // partial index of (split 0, head 0)
+      // weights 2^(lse_s - M) / sum into shared memory [Hq][S]: every (head, split) log-sum-exp
+      // is loaded at once, then one thread per head reduces its S values
+      float* wn = reinterpret_cast<float*>(smem);
+      for (int p = tid; p < Hq * S; p += C::THREADS) {
+        const int hq = p / S, sp = p % S;
+        wn[p] = __ldcg(a.part_lse + b0 + (long long)sp * Hq + hq);
+      }
+      __syncthreads();
+      if (tid < Hq) {
+        float* w = wn + tid * S;
+        float M = -INFINITY, L = 0.f;
+        for (int sp = 0; sp < S; ++sp) M = fmaxf(M, w[sp]);
+        for (int sp = 0; sp < S; ++sp) {
+          const float e = (M != -INFINITY && w[sp] != -INFINITY) ? exp2f(w[sp] - M) : 0.f;
+          w[sp] = e;
+          L += e;
+        }
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+        for (int sp = 0; sp < S; ++sp) w[sp] *= inv;
+        if (a.lse)
+          a.lse[(long long)row * Hq + tid] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+      }
+      __syncthreads();
+      // outputs, 4 head dims per thread: independent 16-byte loads of every split's partial
+      const long long sstride = (long long)Hq * D / 4;  // float4s between splits
+      const float4* part4 = reinterpret_cast<const float4*>(a.part_o) + b0 * D / 4;
+      for (int v = tid; v < Hq * D / 4; v += C::THREADS) {
+        const int hq = (v * 4) / D;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int sp = 0; sp < S; ++sp) {
+          const float w = wn[hq * S + sp];
+          const float4 p = __ldcg(part4 + sp * sstride + v);
+          acc.x = fmaf(w, p.x, acc.x);
+          acc.y = fmaf(w, p.y, acc.y);
+          acc.z = fmaf(w, p.z, acc.z);
+          acc.w = fmaf(w, p.w, acc.w);
+        }
+        uint2 packed;
+        packed.x = pack_bf16(acc.x, acc.y);
+        packed.y = pack_bf16(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(a.out + (long long)row * Hq * D + (long long)v * 4) = packed;
+      }
+      if (tid == 0) a.arrivals[row] = 0u;
     }
   }
 }
@@ -692,9 +755,13 @@ int resolve_sparse_splits(const Geometry& g, int requested) {
   return s;
 }
 
+// Split-K workspace: partial outputs fp32 [num_q, splits, Hq, D], their log2-sum-exp
+// [num_q, splits, Hq], and (swap-AB kernel, Hq/Hkv <= 8) per-row arrival counters [num_q].
 size_t sparse_decode_workspace_bytes(const Geometry& g, int splits) {
+  if (splits <= 1) return 0;
   const size_t n = (size_t)g.num_q * splits * g.Hq;
-  return ((n * g.D * 4 + 255) / 256) * 256 + ((n * 4 + 255) / 256) * 256;
+  return ((n * g.D * 4 + 255) / 256) * 256 + ((n * 4 + 255) / 256) * 256 +
+         (((size_t)g.num_q * 4 + 255) / 256) * 256;
 }
 
 cudaError_t launch_combine(const Geometry& g, const float* part_o, const float* part_lse,
@@ -732,10 +799,16 @@ cudaError_t launch_sparse_attn(const Geometry& g, const void* q, const void* k_p
   a.err = g.err;
   a.part_o = nullptr;
   a.part_lse = nullptr;
+  a.arrivals = nullptr;
   if (splits > 1) {
     const size_t n = (size_t)g.num_q * splits * g.Hq;
     a.part_o = static_cast<float*>(ws);
     a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ((n * g.D * 4 + 255) / 256) * 256);
+    a.arrivals = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.part_lse) + ((n * 4 + 255) / 256) * 256);
+    if (g.G <= 8) {  // the swap-AB kernel merges its splits itself, counting arrivals from zero
+      cudaError_t e = cudaMemsetAsync(a.arrivals, 0, (size_t)g.num_q * 4, s);
+      if (e != cudaSuccess) return e;
+    }
   }
   cudaError_t e;
 #define QSA_SPARSE_CASE(DD, HH) \
@@ -750,7 +823,7 @@ cudaError_t launch_sparse_attn(const Geometry& g, const void* q, const void* k_p
   QSA_SPARSE_CASE(128, 8)
   e = cudaErrorInvalidValue;
 #undef QSA_SPARSE_CASE
-  if (e != cudaSuccess || splits == 1) return e;
+  if (e != cudaSuccess || splits == 1 || g.G <= 8) return e;
   return launch_combine(g, a.part_o, a.part_lse, splits, out, lse, s);
 }
 

@@ -15,10 +15,14 @@
 //    the causal limit, and appends every key above the row's running threshold to a per-row
 //    candidate buffer; a full buffer is cut back to the exact top-k by a warp radix select, which
 //    also raises the threshold.
-//  * materialised (few query rows, e.g. decode with 4 sequences x 4 positions at 1M context): all
-//    SMs split the block range, write fp32 scores (16 MiB, L2-resident), then a histogram of the
-//    top 11 bits of the ordered score finds the bucket holding the k-th score, a filter pass
-//    collects the keys above/in that bucket, and one CTA per row finishes the exact selection.
+//  * materialised (few query rows, any Di): all SMs split the block range, write fp32 scores
+//    (16 MiB at 4 sequences x 4 positions x 1M context, L2-resident), then a histogram of the top
+//    11 bits of the ordered score finds the bucket holding the k-th score, a filter pass collects
+//    the keys above/in that bucket, and one CTA per row finishes the exact selection.
+//  * split lists (few query rows, Di = 128; score_dec.cu): every warp streams a chunk of pages
+//    and keeps each row's 32 best keys of its chunk; one CTA per row merges the lists exactly.
+// The tensor-core (score_tc.cu) and split-list kernels flag rows they cannot settle exactly; the
+// streaming kernel recomputes just those rows.
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
@@ -702,7 +706,9 @@ size_t mat_bytes(const Geometry& g) {
 }  // namespace
 
 int resolve_score_path(const Geometry& g, int requested) {
-  if (requested == 1 || requested == 2) return requested;
+  if (requested == 3 && !score_dec_supported(g)) return 2;
+  if (requested >= 1 && requested <= 3) return requested;
+  if (g.num_q <= 128 && score_dec_supported(g)) return 3;
   return g.num_q <= 256 ? 2 : 1;
 }
 
@@ -712,6 +718,7 @@ size_t score_workspace_bytes(const Geometry& g, int path) {
     if (score_tc_supported(g)) n = std::max(n, score_tc_workspace_bytes(g));
     return n;
   }
+  if (path == 3) return score_dec_workspace_bytes(g);
   return mat_bytes(g);
 }
 
@@ -734,6 +741,12 @@ cudaError_t launch_score_topk(const Geometry& g, int path, const void* idx_q, co
       case 64: return run_stream<64>(a, g, ws, s);
       default: return run_stream<128>(a, g, ws, s);
     }
+  }
+  if (path == 3) {
+    int32_t* redo = nullptr;
+    cudaError_t e = launch_score_dec(a, g, ws, &redo, s);
+    if (e != cudaSuccess) return e;
+    return run_stream<128>(a, g, ws, s, redo);
   }
   MatWs w = carve_mat(g, ws);
   mat_clear_kernel<<<64, 256, 0, s>>>(w, g.num_q);

@@ -1,5 +1,8 @@
 // Pieces shared by the indexer scoring kernels (score.cu, score_tc.cu).
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -97,10 +100,33 @@ inline ScoreArgs make_args(const Geometry& g, const void* idx_q, const void* idx
 }
 
 
+// Tiled TMA loads (tensor map in kernel-parameter space) completing on an mbarrier.
+__device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* m, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+      "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma3d(uint32_t dst, const CUtensorMap* m, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),
+      "l"((uint64_t)m), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// cuTensorMapEncodeTiled from the driver (looked up once), or nullptr.  In score_tc.cu.
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn();
+
 // score_tc.cu: the tcgen05 kernel (Di = 128) used by the streaming path.
 bool score_tc_supported(const Geometry& g);
 size_t score_tc_workspace_bytes(const Geometry& g);
 cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int32_t** redo_out,
                             cudaStream_t s);
+
+// score_dec.cu: decode-sized batches (split warp lists + exact merge; Di = 128).
+bool score_dec_supported(const Geometry& g);
+size_t score_dec_workspace_bytes(const Geometry& g);
+cudaError_t launch_score_dec(const ScoreArgs& a, const Geometry& g, void* ws, int32_t** redo_out,
+                             cudaStream_t s);
 
 }  // namespace qsa

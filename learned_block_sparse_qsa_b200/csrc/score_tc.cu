@@ -27,9 +27,6 @@
 // exactly (radix select on 64-bit keys, lower block index wins ties) with a merge by rank.  Rows
 // that fail the check (adversarial score orders) or overflow the buffer are recomputed by the exact
 // streaming kernel, so the result never depends on the sample.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "common.cuh"
 #include "internal.h"
 #include "score_common.cuh"
@@ -79,18 +76,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_BLK >> 3) << 17) |
                             ((uint32_t)(TC_ROWS >> 4) << 24);
 
-__device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* m, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
-      "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_addr(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tma3d(uint32_t dst, const CUtensorMap* m, int x, int y, int z, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),
-      "l"((uint64_t)m), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
-      : "memory");
-}
 __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t acc) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
@@ -471,7 +456,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+}  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -483,9 +470,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-}  // namespace
-
-bool score_tc_supported(const Geometry& g) { return g.Di == 128 && encode_fn() != nullptr; }
+bool score_tc_supported(const Geometry& g) { return g.Di == 128 && tmap_encode_fn() != nullptr; }
 
 size_t score_tc_workspace_bytes(const Geometry& g) {
   return (size_t)g.num_q * 2 * TC_CAP * 8 + ((size_t)g.num_q * 4 + 255) / 256 * 256;
@@ -495,7 +480,7 @@ size_t score_tc_workspace_bytes(const Geometry& g) {
 // slice) for the exact streaming kernel, which the caller launches next.
 cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int32_t** redo_out,
                             cudaStream_t s) {
-  auto enc = encode_fn();
+  auto enc = tmap_encode_fn();
   if (!enc) return cudaErrorNotSupported;
   u64* cand = static_cast<u64*>(ws);
   int32_t* redo = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + (size_t)g.num_q * 2 * TC_CAP * 8);

@@ -60,13 +60,16 @@ class Run:
         self.torch.cuda.synchronize()
         _ = QsaBatch
 
-    def step(self, decode=None, splits=0):
+    def step(self, decode=None, splits=0, compress=True):
+        """compress=False skips compressing the step's new tokens (for steps whose new tokens do
+        not fill whole blocks; their blocks are never candidates of these rows)."""
         d = self.di
         decode = (self.c.mode == "decode") if decode is None else decode
         kw = dict(q=d.q, idx_q=d.idx_q, idx_w=d.idx_w, kcomp_pool=d.kcomp_pool, k_pool=d.k_pool,
                   v_pool=d.v_pool, out=self.out, sel=self.sel, n_sel=self.n_sel, lse=self.lse,
-                  sel_scores=self.sel_scores, idx_k_new=d.idx_k_new, new_seq=d.new_seq,
-                  new_pos=d.new_pos)
+                  sel_scores=self.sel_scores)
+        if compress:
+            kw.update(idx_k_new=d.idx_k_new, new_seq=d.new_seq, new_pos=d.new_pos)
         if decode:
             self.runner.decode(self.b, splits=splits, **kw)
         else:

@@ -52,7 +52,9 @@ def test_workspace_sizes_are_host_computable():
     n_stream = q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK)
     assert n_stream >= 16384 * 2048 * 8           # streaming path: >= 2048 candidate slots per row
     b = mk_batch(num_q=16, batch=4, max_pages=16384, num_pages=65536, max_pos=1048575)
-    n_mat = q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK)
+    assert q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK) > 0
+    cfg_mat = q.QsaConfig.make(32, 4, 128, 128, score_path=2)
+    n_mat = q.qsa_workspace_size(cfg_mat, b, q.QSA_OP_INDEX_SCORE_TOPK)
     assert n_mat >= 16 * 262144 * 12              # materialised path: scores + boundary keys
     assert q.qsa_workspace_size(cfg, b, q.QSA_OP_SPARSE_ATTN_DECODE, 1) == 0
     assert q.qsa_workspace_size(cfg, b, q.QSA_OP_SPARSE_ATTN_DECODE, 8) >= 16 * 8 * 32 * 129 * 4
@@ -62,7 +64,7 @@ def test_workspace_sizes_are_host_computable():
     ("block_tokens", 8, q.QSA_ERR_UNSUPPORTED), ("idx_heads", 2, q.QSA_ERR_UNSUPPORTED),
     ("head_dim", 96, q.QSA_ERR_UNSUPPORTED), ("topk_blocks", 0, q.QSA_ERR_UNSUPPORTED),
     ("topk_blocks", 513, q.QSA_ERR_UNSUPPORTED), ("num_q_heads", 6, q.QSA_ERR_INVALID_ARG),
-    ("page_tokens", 32, q.QSA_ERR_UNSUPPORTED), ("score_path", 3, q.QSA_ERR_INVALID_ARG)])
+    ("page_tokens", 32, q.QSA_ERR_UNSUPPORTED), ("score_path", 4, q.QSA_ERR_INVALID_ARG)])
 def test_invalid_config_rejected_before_launch(field, value, status):
     cfg = q.QsaConfig.make(32, 4, 128, 128)
     setattr(cfg, field, value)
@@ -89,6 +91,6 @@ def test_invalid_arguments_rejected_before_launch():
         q.qsa_sparse_attn_prefill(cfg, bad, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, stream=0)
     assert e.value.status == q.QSA_ERR_INVALID_ARG
     with pytest.raises(q.QsaError) as e:   # decode with splits but no workspace
-        q.qsa_sparse_attn_decode(cfg, b, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, 4,
+        q.qsa_sparse_attn_decode(cfg, b, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, 12,
                                  None, 0, stream=0)
     assert e.value.status == q.QSA_ERR_WORKSPACE
