@@ -674,25 +674,45 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
           a.lse[(long long)row * Hq + tid] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
       }
       __syncthreads();
-      // outputs, 4 head dims per thread: independent 16-byte loads of every split's partial
+      // outputs: each thread owns up to 4 float4 groups of head dims and walks the splits once,
+      // so that 4 independent 16-byte loads per split (12 with the unrolling) are in flight
+      constexpr int VPT = 4;
       const long long sstride = (long long)Hq * D / 4;  // float4s between splits
       const float4* part4 = reinterpret_cast<const float4*>(a.part_o) + b0 * D / 4;
-      for (int v = tid; v < Hq * D / 4; v += C::THREADS) {
-        const int hq = (v * 4) / D;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int sp = 0; sp < S; ++sp) {
-          const float w = wn[hq * S + sp];
-          const float4 p = __ldcg(part4 + sp * sstride + v);
-          acc.x = fmaf(w, p.x, acc.x);
-          acc.y = fmaf(w, p.y, acc.y);
-          acc.z = fmaf(w, p.z, acc.z);
-          acc.w = fmaf(w, p.w, acc.w);
+      const int nv = Hq * D / 4;
+      for (int v0 = tid; v0 < nv; v0 += VPT * C::THREADS) {
+        float4 acc[VPT];
+        int hqv[VPT];
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+          acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          hqv[j] = (v0 + j * C::THREADS) * 4 / D;
         }
-        uint2 packed;
-        packed.x = pack_bf16(acc.x, acc.y);
-        packed.y = pack_bf16(acc.z, acc.w);
-        *reinterpret_cast<uint2*>(a.out + (long long)row * Hq * D + (long long)v * 4) = packed;
+#pragma unroll 3
+        for (int sp = 0; sp < S; ++sp) {
+#pragma unroll
+          for (int j = 0; j < VPT; ++j) {
+            const int v = v0 + j * C::THREADS;
+            if (v < nv) {
+              const float w = wn[hqv[j] * S + sp];
+              const float4 p = __ldcg(part4 + sp * sstride + v);
+              acc[j].x = fmaf(w, p.x, acc[j].x);
+              acc[j].y = fmaf(w, p.y, acc[j].y);
+              acc[j].z = fmaf(w, p.z, acc[j].z);
+              acc[j].w = fmaf(w, p.w, acc[j].w);
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+          const int v = v0 + j * C::THREADS;
+          if (v < nv) {
+            uint2 packed;
+            packed.x = pack_bf16(acc[j].x, acc[j].y);
+            packed.y = pack_bf16(acc[j].z, acc[j].w);
+            *reinterpret_cast<uint2*>(a.out + (long long)row * Hq * D + (long long)v * 4) = packed;
+          }
+        }
       }
       if (tid == 0) a.arrivals[row] = 0u;
     }

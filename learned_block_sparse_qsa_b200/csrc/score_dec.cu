@@ -48,7 +48,8 @@ constexpr int DS_CTA_MERGE_W = 512; // from this many warp chunks on, CTAs merge
 constexpr int DS_PAGE = 16 * 128 * 2;  // one page of compressed keys, Di = 128
 constexpr int DM_THREADS = 512;
 constexpr int DM_MAXU = 8192;       // keys in one row's union
-static_assert(DM_THREADS == 512, "the merge sorts one selected block per thread");
+static_assert(DM_THREADS == 512 && 2 * DM_THREADS >= DS_MAXW,
+              "16 warps; the list-offset scan takes two lists per thread");
 static_assert(DS_MAXW / DS_WARPS * DS_KC <= DM_MAXU && (DS_CTA_MERGE_W - 1) * DS_KW <= DM_MAXU,
               "union bound");
 
@@ -426,12 +427,16 @@ __global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
 
 // ------------------------------------------------------------------ merge (one CTA per row)
 
+constexpr int DM_CAND = 512;  // keys of the boundary histogram bin ranked directly
+
 struct MergeSmem {
   static constexpr int KEYS = DM_MAXU * 8;
   static constexpr int BOUNDS = DS_MAXW * 8;
   static constexpr int HIST = 2048 * 4;
-  static constexpr int XCH = DM_THREADS * 8;  // bitonic exchange
-  static constexpr int TOTAL = KEYS + BOUNDS + HIST + XCH + 256;
+  static constexpr int CAND = DM_CAND * 8;
+  static constexpr int LISTS = 2 * DS_MAXW * 4;  // selected count and output offset per list
+  static constexpr int TAIL = 640;  // reductions, barrier, scan totals, selection scalars
+  static constexpr int TOTAL = KEYS + BOUNDS + HIST + CAND + LISTS + TAIL;
 };
 
 // Exclusive prefix sum over the CTA (DM_THREADS threads); wsum: 32 words of shared memory.
@@ -562,45 +567,29 @@ __device__ u64 cta_kth_largest(const u64* keys, int n, int need, uint32_t* hist,
   }
 }
 
-// Sort one 64-bit value per thread ascending over the CTA (DM_THREADS = 512): bitonic network,
-// exchanges at distance >= 32 through shared memory, shorter ones by warp shuffles.
-__device__ __forceinline__ u64 cta_sort_asc(u64 v, u64* xch) {
-  const int tid = threadIdx.x;
-#pragma unroll 1
-  for (int k = 2; k <= DM_THREADS; k <<= 1) {
-#pragma unroll 1
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      u64 o;
-      if (j >= 32) {
-        xch[tid] = v;
-        __syncthreads();
-        o = xch[tid ^ j];
-        __syncthreads();
-      } else {
-        o = __shfl_xor_sync(0xffffffffu, v, j);
-      }
-      const bool take_min = ((tid & j) == 0) == ((tid & k) == 0);
-      v = take_min ? (o < v ? o : v) : (o > v ? o : v);
-    }
-  }
-  return v;
-}
-
+// One CTA per query row.  The row's lists come in block order (list l covers a block range below
+// list l+1's) and each is sorted by key, so the need keys >= tau are a prefix of every list: the
+// output is the lists' prefixes in list order, each put in block order by a warp-level rank.
 __global__ void __launch_bounds__(DM_THREADS)
     dec_merge_kernel(ScoreArgs a, DecWs ws, int nl, int lk) {
   extern __shared__ __align__(128) uint8_t smem[];
   u64* keys = reinterpret_cast<u64*>(smem);
   u64* bnds = reinterpret_cast<u64*>(smem + MergeSmem::KEYS);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + MergeSmem::KEYS + MergeSmem::BOUNDS);
-  u64* xch = reinterpret_cast<u64*>(smem + MergeSmem::KEYS + MergeSmem::BOUNDS + MergeSmem::HIST);
-  uint8_t* tail = smem + MergeSmem::KEYS + MergeSmem::BOUNDS + MergeSmem::HIST + MergeSmem::XCH;
-  u64* red = reinterpret_cast<u64*>(tail);                     // [16] per-warp reductions
-  uint64_t* bar = reinterpret_cast<uint64_t*>(tail + 128);     // bulk-copy barrier
-  uint32_t* wsum = reinterpret_cast<uint32_t*>(tail + 136);    // [16] scan totals
-  uint32_t* sel3 = reinterpret_cast<uint32_t*>(tail + 200);    // [3] digit, above, count
-  int* s_n = reinterpret_cast<int*>(tail + 212);
+  u64* cand = reinterpret_cast<u64*>(smem + MergeSmem::KEYS + MergeSmem::BOUNDS + MergeSmem::HIST);
+  int* lcnt = reinterpret_cast<int*>(smem + MergeSmem::KEYS + MergeSmem::BOUNDS + MergeSmem::HIST +
+                                     MergeSmem::CAND);
+  int* loff = lcnt + DS_MAXW;
+  uint8_t* tail = reinterpret_cast<uint8_t*>(loff + DS_MAXW);
+  u64* red = reinterpret_cast<u64*>(tail);                    // [3][16] per-warp min, max, bound
+  uint32_t* redn = reinterpret_cast<uint32_t*>(tail + 384);  // [16] per-warp kept counts
+  uint64_t* bar = reinterpret_cast<uint64_t*>(tail + 448);
+  uint32_t* wsum = reinterpret_cast<uint32_t*>(tail + 456);  // [16] scan totals
+  uint32_t* sel3 = reinterpret_cast<uint32_t*>(tail + 520);  // digit, above, count, n in bin
+  u64* s_tau = reinterpret_cast<u64*>(tail + 536);
 
-  const int row = blockIdx.x, tid = threadIdx.x, warp = tid >> 5;
+  const int row = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int NW = DM_THREADS / 32;
   const int seq = a.q_seq[row], pos = a.q_pos[row];
   const bool ok = seq >= 0 && seq < a.batch && pos >= 0 && pos / 64 < a.max_pages && pos <= a.max_pos;
   if (!ok) {  // already flagged by the score kernel
@@ -612,11 +601,12 @@ __global__ void __launch_bounds__(DM_THREADS)
   const int need = min(a.topk, lim);
   int32_t* srow = a.sel + (long long)row * a.sel_stride;
   float* crow = a.sel_scores ? a.sel_scores + (long long)row * a.sel_stride : nullptr;
+  // the tail block and the padding after the need selected blocks
+  for (int i = need + tid; i < a.sel_stride; i += DM_THREADS) {
+    srow[i] = i == need ? lim : -1;
+    if (crow) crow[i] = i == need ? __int_as_float(0x7f800000) : __int_as_float(0x7fc00000);
+  }
   if (need == 0) {
-    for (int i = tid; i < a.sel_stride; i += DM_THREADS) {
-      srow[i] = i == 0 ? lim : -1;
-      if (crow) crow[i] = i == 0 ? __int_as_float(0x7f800000) : __int_as_float(0x7fc00000);
-    }
     if (tid == 0) {
       a.n_sel[row] = 1;
       ws.redo[row] = 0;
@@ -642,52 +632,147 @@ __global__ void __launch_bounds__(DM_THREADS)
     if (tid == 0) ws.redo[row] = 1;
     return;
   }
-  // kept keys in all, and the largest bound: every key a list dropped lies below it
-  uint32_t nkept = 0;
-  for (int i = tid; i < U; i += DM_THREADS) nkept += keys[i] != 0ull;
-  u64 maxb = 0;
-  for (int i = tid; i < nl; i += DM_THREADS) maxb = bnds[i] > maxb ? bnds[i] : maxb;
-  const u64 maxmin = cta_max_u64(maxb, red);
-  nkept = cta_excl_scan(nkept, wsum) + nkept;  // inclusive; the last thread holds the total
-  if (tid == DM_THREADS - 1) *s_n = (int)nkept;
-  __syncthreads();
-  bool exact = *s_n >= need;
-  __syncthreads();
-  u64 tau = 0;
-  if (exact) {
-    tau = cta_kth_largest(keys, U, need, hist, red, wsum, sel3);
-    exact = maxmin <= tau;
+
+  // one pass: kept keys, smallest kept and largest key, and the largest bound (every key a list
+  // dropped lies below its bound), reduced per warp and then by every thread from 16 entries
+  uint32_t nk = 0;
+  u64 lo = ~0ull, hi = 0ull, mb = 0ull;
+  for (int i = tid; i < U; i += DM_THREADS) {
+    const u64 k = keys[i];
+    if (k) {
+      ++nk;
+      lo = k < lo ? k : lo;
+      hi = k > hi ? k : hi;
+    }
   }
-  if (!exact) {  // the exact streaming kernel recomputes this row
+  for (int i = tid; i < nl; i += DM_THREADS) mb = bnds[i] > mb ? bnds[i] : mb;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    nk += __shfl_xor_sync(0xffffffffu, nk, o);
+    const u64 x = __shfl_xor_sync(0xffffffffu, lo, o), y = __shfl_xor_sync(0xffffffffu, hi, o),
+              z = __shfl_xor_sync(0xffffffffu, mb, o);
+    lo = x < lo ? x : lo;
+    hi = y > hi ? y : hi;
+    mb = z > mb ? z : mb;
+  }
+  if (lane == 0) {
+    red[warp] = lo;
+    red[16 + warp] = hi;
+    red[32 + warp] = mb;
+    redn[warp] = nk;
+  }
+  __syncthreads();
+  nk = 0;
+  lo = ~0ull;
+  hi = 0ull;
+  mb = 0ull;
+  for (int w = 0; w < NW; ++w) {
+    nk += redn[w];
+    lo = red[w] < lo ? red[w] : lo;
+    hi = red[16 + w] > hi ? red[16 + w] : hi;
+    mb = red[32 + w] > mb ? red[32 + w] : mb;
+  }
+  if ((int)nk < need) {  // lists dropped too much: the exact kernel redoes the row
     if (tid == 0) ws.redo[row] = 1;
     return;
   }
-  // the need keys >= tau, packed (block : score bits) and sorted by block
-  if (tid == 0) *s_n = 0;
-  __syncthreads();
-  u64* packed = reinterpret_cast<u64*>(hist);  // 512 x 8 B over the free histogram
-  for (int i = tid; i < U; i += DM_THREADS) {
-    const u64 k = keys[i];
-    if (k >= tau) packed[atomicAdd(s_n, 1)] = ((u64)key_block(k) << 32) | __float_as_uint(key_score(k));
+
+  // tau = the need-th largest kept key: one CTA histogram of 11 bits below the highest bit where
+  // the kept keys differ, then the few keys of the boundary bin are ranked directly
+  u64 tau;
+  if ((int)nk == need) {
+    tau = lo;
+  } else {
+    const int top = 63 - __clzll((long long)(lo ^ hi));
+    const int width = top + 1 < 11 ? top + 1 : 11;
+    const int shift = top + 1 - width;
+    const uint32_t nb = 1u << width;
+    const u64 hmask = top < 63 ? ~((2ull << top) - 1ull) : 0ull;  // bits every kept key shares
+    const u64 prefix = hi & hmask;
+    for (uint32_t i = tid; i < nb; i += DM_THREADS) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < U; i += DM_THREADS) {
+      const u64 k = keys[i];
+      if (k && (k & hmask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    const int per = (int)(nb + DM_THREADS - 1) / DM_THREADS;  // bins per thread from the top
+    uint32_t tot = 0;
+    for (int j = 0; j < per; ++j) {
+      const int bin = (int)nb - 1 - (tid * per + j);
+      if (bin >= 0) tot += hist[bin];
+    }
+    const uint32_t excl = cta_excl_scan(tot, wsum);
+    if (excl < (uint32_t)need && (uint32_t)need <= excl + tot) {
+      uint32_t acc = excl;
+      for (int j = 0; j < per; ++j) {
+        const int bin = (int)nb - 1 - (tid * per + j);
+        const uint32_t c = hist[bin];
+        if (acc + c >= (uint32_t)need) {
+          sel3[0] = (uint32_t)bin;
+          sel3[1] = acc;  // kept keys in higher bins
+          sel3[2] = c;
+          break;
+        }
+        acc += c;
+      }
+    }
+    if (tid == 0) sel3[3] = 0;
+    __syncthreads();
+    const uint32_t digit = sel3[0], above = sel3[1], inbin = sel3[2];
+    if (inbin <= (uint32_t)DM_THREADS) {
+      // the boundary bin's keys, each ranked by counting the larger ones (keys are unique)
+      const u64 bmask = hmask | ((u64)(nb - 1) << shift);
+      const u64 bpre = prefix | ((u64)digit << shift);
+      for (int i = tid; i < U; i += DM_THREADS) {
+        const u64 k = keys[i];
+        if (k && (k & bmask) == bpre) cand[atomicAdd(&sel3[3], 1u)] = k;
+      }
+      __syncthreads();
+      if (tid < (int)inbin) {
+        const u64 k = cand[tid];
+        uint32_t r = 0;
+        for (uint32_t j = 0; j < inbin; ++j) r += cand[j] > k;
+        if (r == (uint32_t)need - above - 1u) *s_tau = k;
+      }
+      __syncthreads();
+      tau = *s_tau;
+    } else {  // a crowded bin: the full CTA radix select
+      tau = cta_kth_largest(keys, U, need, hist, red, wsum, sel3);
+    }
+  }
+  if (mb > tau) {  // a dropped key could beat tau: the exact kernel redoes the row
+    if (tid == 0) ws.redo[row] = 1;
+    return;
+  }
+
+  // keys >= tau per list (a prefix: lists are sorted by key), then each list's output offset
+  for (int w = warp; w < nl; w += NW) {
+    const bool sel = lane < lk && keys[w * lk + lane] >= tau;
+    const int c = __popc(__ballot_sync(0xffffffffu, sel));
+    if (lane == 0) lcnt[w] = c;
   }
   __syncthreads();
-  u64 v = tid < need ? packed[tid] : ~0ull;
-  v = cta_sort_asc(v, xch);
-  for (int i = tid; i < a.sel_stride; i += DM_THREADS) {
-    int32_t b;
-    float sc;
-    if (i < need) {  // i == tid here (need <= 512)
-      b = (int32_t)(v >> 32);
-      sc = __uint_as_float((uint32_t)v);
-    } else if (i == need) {
-      b = lim;                          // the tail block
-      sc = __int_as_float(0x7f800000);  // +inf marks it
-    } else {
-      b = -1;
-      sc = __int_as_float(0x7fc00000);
+  {
+    int c0 = 2 * tid < nl ? lcnt[2 * tid] : 0, c1 = 2 * tid + 1 < nl ? lcnt[2 * tid + 1] : 0;
+    const uint32_t ex = cta_excl_scan((uint32_t)(c0 + c1), wsum);
+    if (2 * tid < nl) loff[2 * tid] = (int)ex;
+    if (2 * tid + 1 < nl) loff[2 * tid + 1] = (int)ex + c0;
+  }
+  __syncthreads();
+  // each list's selected keys in block order: rank by comparison within the prefix
+  for (int w = warp; w < nl; w += NW) {
+    const int c = lcnt[w];
+    if (c == 0) continue;
+    const u64 k = lane < c ? keys[w * lk + lane] : 0ull;
+    const uint32_t b = lane < c ? key_block(k) : 0xFFFFFFFFu;
+    int r = 0;
+    for (int j = 0; j < c; ++j) r += __shfl_sync(0xffffffffu, b, j) < b;
+    if (lane < c) {
+      const int o = loff[w] + r;
+      srow[o] = (int32_t)b;
+      if (crow) crow[o] = key_score(k);
     }
-    srow[i] = b;
-    if (crow) crow[i] = sc;
   }
   if (tid == 0) {
     a.n_sel[row] = need + 1;
