@@ -76,6 +76,31 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_BLK >> 3) << 17) |
                             ((uint32_t)(TC_ROWS >> 4) << 24);
 
+// Packed fp32 pairs (sm_100): one instruction rounds both lanes exactly as the scalar op would.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t acc) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
@@ -308,7 +333,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           if (dead) return false;
           tc_fence_after();
-          const float wa = w[pair * 2], wb = w[pair * 2 + 1];
+          // two blocks per packed fp32x2 multiply / fma / add: wb*relu(vb) + wa*relu(va), the same
+          // rounding steps as the scalar fmaf(wb, relu(vb), wa * relu(va))
+          const uint64_t wa2 = pack_f32x2(w[pair * 2], w[pair * 2]);
+          const uint64_t wb2 = pack_f32x2(w[pair * 2 + 1], w[pair * 2 + 1]);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             float va[16], vb[16];
@@ -317,9 +345,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tmem_ld16(col + TC_BLK, vb);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float x = fmaf(wb, fmaxf(vb[j], 0.f), wa * fmaxf(va[j], 0.f));
-              sc[c * 16 + j] = pair == 0 ? x : sc[c * 16 + j] + x;
+            for (int j = 0; j < 16; j += 2) {
+              const uint64_t ra = pack_f32x2(fmaxf(va[j], 0.f), fmaxf(va[j + 1], 0.f));
+              const uint64_t rb = pack_f32x2(fmaxf(vb[j], 0.f), fmaxf(vb[j + 1], 0.f));
+              uint64_t x = fma_f32x2(wb2, rb, mul_f32x2(wa2, ra));
+              if (pair == 1) x = add_f32x2(pack_f32x2(sc[c * 16 + j], sc[c * 16 + j + 1]), x);
+              unpack_f32x2(x, sc[c * 16 + j], sc[c * 16 + j + 1]);
             }
           }
           tc_fence_before();
