@@ -175,6 +175,7 @@ def qsa_dense_attn_decode(cfg, batch, q, k_pool, v_pool, out, lse, num_splits, w
            "qsa_dense_attn_decode")
 
 
-from .runner import QsaRunner  # noqa: E402  (sequences the calls above; owns workspaces)
+from .runner import BlockCarry, QsaRunner, compress_split  # noqa: E402  (step sequencing)
 
-__all__ = [n for n in list(globals()) if n.startswith(("qsa_", "Qsa", "QSA_"))] + ["DEVERR", "LIB_PATH"]
+__all__ = [n for n in list(globals()) if n.startswith(("qsa_", "Qsa", "QSA_"))] + [
+    "DEVERR", "LIB_PATH", "BlockCarry", "compress_split"]

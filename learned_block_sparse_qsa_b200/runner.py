@@ -20,6 +20,51 @@ from . import (QSA_OP_DENSE_ATTN_DECODE, QSA_OP_INDEX_SCORE_TOPK, QSA_OP_SPARSE_
                qsa_sparse_attn_prefill, qsa_workspace_size)
 
 
+def compress_split(carry_pos: int, carry_len: int, pos0: int, n_new: int):
+    """How one prefill chunk of a sequence feeds step (a) when chunk boundaries are not multiples
+    of the 4-token block (the article's "unfinished block at the sequence tail" carries over).
+
+    carry_pos, carry_len: the carried raw keys cover positions [carry_pos, carry_pos + carry_len)
+    of the block that the previous chunk left unfinished (carry_len in 0..3).  The chunk's new
+    keys cover [pos0, pos0 + n_new) and must continue the carry.  Returns (start, n_compress,
+    next_carry_pos, next_carry_len): the keys [start, start + n_compress) -- carry first, then the
+    chunk's -- form whole blocks to compress now, and the rest is carried to the next chunk."""
+    if carry_len:
+        if carry_pos % 4 or carry_pos + carry_len != pos0:
+            raise ValueError("the chunk must continue the carried block")
+        start = carry_pos
+    else:
+        if pos0 % 4:
+            raise ValueError("a chunk that starts inside a block needs that block's earlier keys")
+        start = pos0
+    total = (pos0 + n_new) - start
+    n_compress = total // 4 * 4
+    return start, n_compress, start + n_compress, total - n_compress
+
+
+class BlockCarry:
+    """Per-sequence raw indexer keys of the unfinished block, carried between prefill chunks so
+    that every block is compressed exactly once, when it completes.  Device tensors only; the
+    compression itself is qsa_index_compress."""
+
+    def __init__(self):
+        self._carry: dict[int, tuple[int, torch.Tensor]] = {}
+
+    def compress_chunk(self, runner: "QsaRunner", b: QsaBatch, seq: int, pos0: int, idx_k_new,
+                       kcomp_pool, stream=None):
+        """Compress the blocks that the chunk's keys idx_k_new ([n, Di], positions pos0..) complete."""
+        cpos, ckeys = self._carry.get(seq, (pos0, idx_k_new[:0]))
+        start, n, npos, nlen = compress_split(cpos, ckeys.shape[0], pos0, idx_k_new.shape[0])
+        keys = torch.cat([ckeys, idx_k_new]) if ckeys.shape[0] else idx_k_new
+        if n:
+            dev = keys.device
+            seqs = torch.full((n,), seq, dtype=torch.int32, device=dev)
+            poss = torch.arange(start, start + n, dtype=torch.int32, device=dev)
+            runner.compress(b, keys[:n].contiguous(), seqs, poss, kcomp_pool, stream)
+        self._carry[seq] = (npos, keys[n:].clone())
+        return n
+
+
 class QsaRunner:
     def __init__(self, cfg: QsaConfig, device="cuda"):
         self.cfg = cfg
@@ -89,4 +134,4 @@ class QsaRunner:
         self.err.zero_()
 
 
-__all__ = ["QsaRunner", "ctypes"]
+__all__ = ["QsaRunner", "BlockCarry", "compress_split", "ctypes"]
