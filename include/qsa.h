@@ -188,6 +188,14 @@ qsa_status_t qsa_dense_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* b
                                    void* out, float* lse, int32_t num_splits, void* workspace,
                                    size_t ws_bytes, qsa_stream_t stream);
 
+/* No counterpart in the article: a self-test of failure detection.  Every pipelined kernel waits
+ * on mbarriers with a bounded wait that, when it runs out, sets QSA_DEVERR_TIMEOUT in *err_flag
+ * and lets the kernel return instead of hanging.  This call launches one CTA that waits, with that
+ * same helper, on a phase that nothing completes, for limit_cycles (1e3..1e9 SM cycles; outside
+ * that range QSA_ERR_INVALID_ARG): afterwards *err_flag has QSA_DEVERR_TIMEOUT set and the stream
+ * and context remain usable. */
+qsa_status_t qsa_selftest_wait_timeout(int32_t* err_flag, int64_t limit_cycles, qsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

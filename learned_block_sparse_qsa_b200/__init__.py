@@ -90,6 +90,7 @@ _SIGS = {
                                          c_void_p]),
     "qsa_dense_attn_decode": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_int32, c_void_p, c_size_t, c_void_p]),
+    "qsa_selftest_wait_timeout": (c_int32, [c_void_p, c_int64, c_void_p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -173,6 +174,12 @@ def qsa_dense_attn_decode(cfg, batch, q, k_pool, v_pool, out, lse, num_splits, w
                                       _p(v_pool), _p(out), _p(lse), int(num_splits), _p(workspace),
                                       int(ws_bytes), _stream(stream)),
            "qsa_dense_attn_decode")
+
+
+def qsa_selftest_wait_timeout(err_flag, limit_cycles, stream=None):
+    """Launch the bounded-wait self-test (sets QSA_DEVERR_TIMEOUT in err_flag; see include/qsa.h)."""
+    _check(_lib.qsa_selftest_wait_timeout(_p(err_flag), int(limit_cycles), _stream(stream)),
+           "qsa_selftest_wait_timeout")
 
 
 from .runner import BlockCarry, QsaRunner, compress_split  # noqa: E402  (step sequencing)

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/qsa.h"
 
 namespace qsa {
@@ -25,6 +27,8 @@ inline cudaError_t set_smem_once(const void* kernel, int bytes) {
   };
   static Entry table[64];
   static int used = 0;
+  static std::mutex lock;  // host threads may launch on their own streams concurrently
+  std::lock_guard<std::mutex> guard(lock);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const unsigned long long bit = 1ull << (dev & 63);
@@ -115,11 +119,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait: true when the phase completed, false (and QSA_DEVERR_TIMEOUT) after the limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err,
+                                          long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       flag_error(err, QSA_DEVERR_TIMEOUT);
       return false;
     }

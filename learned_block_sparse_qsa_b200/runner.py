@@ -99,22 +99,24 @@ class QsaRunner:
     def prefill(self, b: QsaBatch, *, q, idx_q, idx_w, kcomp_pool, k_pool, v_pool, out, sel, n_sel,
                 idx_k_new=None, new_seq=None, new_pos=None, lse=None, sel_scores=None, stream=None):
         """Whole prefill step: compress (if new keys are given) -> score/select -> attention."""
-        if idx_k_new is not None:
-            self.compress(b, idx_k_new, new_seq, new_pos, kcomp_pool, stream)
-        self.select(b, idx_q, idx_w, kcomp_pool, sel, n_sel, sel_scores, stream)
-        qsa_sparse_attn_prefill(self.cfg, b, q, k_pool, v_pool, sel, n_sel, out, lse, stream)
+        with torch.cuda.nvtx.range("qsa.prefill"):
+            if idx_k_new is not None:
+                self.compress(b, idx_k_new, new_seq, new_pos, kcomp_pool, stream)
+            self.select(b, idx_q, idx_w, kcomp_pool, sel, n_sel, sel_scores, stream)
+            qsa_sparse_attn_prefill(self.cfg, b, q, k_pool, v_pool, sel, n_sel, out, lse, stream)
         return out
 
     def decode(self, b: QsaBatch, *, q, idx_q, idx_w, kcomp_pool, k_pool, v_pool, out, sel, n_sel,
                idx_k_new=None, new_seq=None, new_pos=None, lse=None, sel_scores=None, splits=0,
                stream=None):
         """Whole decode step: compress the new block -> score/select -> split-K attention."""
-        if idx_k_new is not None:
-            self.compress(b, idx_k_new, new_seq, new_pos, kcomp_pool, stream)
-        self.select(b, idx_q, idx_w, kcomp_pool, sel, n_sel, sel_scores, stream)
-        ws, n = self.workspace(b, QSA_OP_SPARSE_ATTN_DECODE, splits)
-        qsa_sparse_attn_decode(self.cfg, b, q, k_pool, v_pool, sel, n_sel, out, lse, splits, ws, n,
-                               stream)
+        with torch.cuda.nvtx.range("qsa.decode"):
+            if idx_k_new is not None:
+                self.compress(b, idx_k_new, new_seq, new_pos, kcomp_pool, stream)
+            self.select(b, idx_q, idx_w, kcomp_pool, sel, n_sel, sel_scores, stream)
+            ws, n = self.workspace(b, QSA_OP_SPARSE_ATTN_DECODE, splits)
+            qsa_sparse_attn_decode(self.cfg, b, q, k_pool, v_pool, sel, n_sel, out, lse, splits,
+                                   ws, n, stream)
         return out
 
     def dense(self, b: QsaBatch, *, q, k_pool, v_pool, out, lse=None, decode=False, splits=0,

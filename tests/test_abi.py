@@ -94,3 +94,12 @@ def test_invalid_arguments_rejected_before_launch():
         q.qsa_sparse_attn_decode(cfg, b, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, 12,
                                  None, 0, stream=0)
     assert e.value.status == q.QSA_ERR_WORKSPACE
+
+
+def test_selftest_rejects_limits_outside_range_before_launch():
+    with pytest.raises(q.QsaError) as e:
+        q.qsa_selftest_wait_timeout(0x1000, 10, stream=0)
+    assert e.value.status == q.QSA_ERR_INVALID_ARG
+    with pytest.raises(q.QsaError) as e:
+        q.qsa_selftest_wait_timeout(None, 1_000_000, stream=0)
+    assert e.value.status == q.QSA_ERR_INVALID_ARG
