@@ -290,84 +290,139 @@ def graph_decode_us(w: Workload, steps: int, warmup: int, flush):
     return statistics.mean(us), us
 
 
+class Staging:
+    """One pinned host buffer holding every per-step input of a workload, and device buffers it is
+    copied into with a single host-to-device copy; tensors are 256-byte aligned views."""
+
+    def __init__(self, torch, host_tensors: dict, copies: int, device):
+        self.torch = torch
+        self.layout, off = {}, 0
+        for name, t in host_tensors.items():
+            n = t.numel() * t.element_size()
+            self.layout[name] = (off, t.dtype, tuple(t.shape), n)
+            off += (n + 255) // 256 * 256
+        self.nbytes = off
+        self.host = torch.empty(off, dtype=torch.uint8).pin_memory()
+        for name, t in host_tensors.items():
+            o, _, _, n = self.layout[name]
+            self.host[o:o + n].copy_(t.contiguous().view(-1).view(torch.uint8))
+        self.dev = [torch.empty(off, dtype=torch.uint8, device=device) for _ in range(copies)]
+
+    def view(self, i: int, name: str):
+        o, dt, shape, n = self.layout[name]
+        return self.dev[i][o:o + n].view(dt).view(shape)
+
+    def h2d(self, i: int):
+        self.dev[i].copy_(self.host, non_blocking=True)
+
+
 def e2e_prefill(w: Workload, steps: int, warmup: int):
-    """Whole step through the public API with host inputs: H2D of the chunk's inputs (queries,
-    indexer queries/weights/keys, the new K/V pages), the layer, D2H of the output."""
+    """Whole step through the public API with host inputs: one host-to-device copy of the chunk's
+    inputs (queries, indexer queries/weights/keys, the new K/V pages), the new pages scattered into
+    the cache, the layer, one device-to-host copy of the output.  Successive steps are pipelined:
+    step k+1's inputs travel (own stream, double buffer) while step k computes, and step k's
+    output travels back (own stream) while step k+1 computes."""
     torch = w.torch
-    c, d = w.c, w.di
-    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    hq, hiq, hiw, hik = pin(d.q), pin(d.idx_q), pin(d.idx_w), pin(d.idx_k_new)
+    c, d, r, b = w.c, w.di, w.runner, w.b
     lp0, lp1 = c.ctx_start // 64, (c.ctx - 1) // 64 + 1
     pages = d.page_table[0, lp0:lp1].long()
-    hk, hv = pin(d.k_pool[pages]), pin(d.v_pool[pages])
-    pages_h = pages.cpu().tolist()
+    st = Staging(torch, {"q": d.q.cpu(), "idx_q": d.idx_q.cpu(), "idx_w": d.idx_w.cpu(),
+                         "idx_k": d.idx_k_new.cpu(), "k": d.k_pool[pages].cpu(),
+                         "v": d.v_pool[pages].cpu()}, 2, d.q.device)
+    outs = [torch.empty_like(d.q) for _ in range(2)]
     hout = torch.empty(d.q.shape, dtype=d.q.dtype).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hiq, hiw, hik, hk, hv))
-    d2h = hout.numel() * hout.element_size()
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        d.q.copy_(hq, non_blocking=True)
-        d.idx_q.copy_(hiq, non_blocking=True)
-        d.idx_w.copy_(hiw, non_blocking=True)
-        d.idx_k_new.copy_(hik, non_blocking=True)
-        for i, p in enumerate(pages_h):
-            d.k_pool[p].copy_(hk[i], non_blocking=True)
-            d.v_pool[p].copy_(hv[i], non_blocking=True)
-        w.step(False)
-        hout.copy_(w.out, non_blocking=True)
+    def run(n):
+        for k in range(n):
+            i = k % 2
+            with torch.cuda.stream(s_in):
+                if k >= 2:
+                    s_in.wait_event(ev_done[i])  # step k-2 is done with staging buffer i
+                st.h2d(i)
+                ev_in[i].record(s_in)
+            comp.wait_event(ev_in[i])
+            if k >= 2:
+                comp.wait_event(ev_out[i])       # step k-2's output has left outs[i]
+            d.k_pool.index_copy_(0, pages, st.view(i, "k"))
+            d.v_pool.index_copy_(0, pages, st.view(i, "v"))
+            r.prefill(b, q=st.view(i, "q"), idx_q=st.view(i, "idx_q"), idx_w=st.view(i, "idx_w"),
+                      kcomp_pool=d.kcomp_pool, k_pool=d.k_pool, v_pool=d.v_pool, out=outs[i],
+                      sel=w.sel, n_sel=w.n_sel, idx_k_new=st.view(i, "idx_k"), new_seq=d.new_seq,
+                      new_pos=d.new_pos)
+            ev_done[i].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[i])
+                hout.copy_(outs[i], non_blocking=True)
+                ev_out[i].record(s_out)
 
-    for _ in range(warmup):
-        one()
+    run(warmup)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        one()
-    b.record()
+    e = torch.cuda.Event(enable_timing=True)
+    a.record(s_in)
+    run(steps)
+    e.record(s_out)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    return ms, h2d, d2h
+    ms = a.elapsed_time(e) / steps
+    # the pipelined result must be the layer's: compare with one plain device step
+    w.step(False)
+    torch.cuda.synchronize()
+    if not torch.equal(hout.view(torch.int16), w.out.cpu().view(torch.int16)):
+        raise RuntimeError("end-to-end prefill output differs from the device step's output")
+    d2h = hout.numel() * hout.element_size()
+    return ms, st.nbytes, d2h
 
 
 def e2e_decode(w: Workload, steps: int, warmup: int):
+    """Whole decode step through the public API with host inputs: one host-to-device copy of the
+    step's inputs (queries, indexer tensors, the new tokens' K/V rows), the rows scattered into the
+    cache, the layer, one device-to-host copy of the output every step."""
     torch = w.torch
     c, d = w.c, w.di
-    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    hq, hiq, hiw, hik = pin(d.q), pin(d.idx_q), pin(d.idx_w), pin(d.idx_k_new)
-    q_pos = d.q_pos.cpu().long()
-    q_seq = d.q_seq.cpu().long()
-    pages = d.page_table.cpu()[q_seq, q_pos // 64].long()
+    q_pos = d.q_pos.long()
+    q_seq = d.q_seq.long()
+    pages = d.page_table[q_seq, q_pos // 64].long()
     slots = (q_pos % 64).long()
-    hk = pin(d.k_pool[pages.cuda(), slots.cuda()])
-    hv = pin(d.v_pool[pages.cuda(), slots.cuda()])
-    kv_dst = list(zip(pages.tolist(), slots.tolist()))
+    st = Staging(torch, {"q": d.q.cpu(), "idx_q": d.idx_q.cpu(), "idx_w": d.idx_w.cpu(),
+                         "idx_k": d.idx_k_new.cpu(), "k": d.k_pool[pages, slots].cpu(),
+                         "v": d.v_pool[pages, slots].cpu()}, 1, d.q.device)
     hout = torch.empty(d.q.shape, dtype=d.q.dtype).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hiq, hiw, hik, hk, hv))
-    d2h = hout.numel() * hout.element_size()
+    from learned_block_sparse_qsa_b200 import QSA_OP_SPARSE_ATTN_DECODE, qsa_sparse_attn_decode
+
+    r, b, cfg = w.runner, w.b, w.cfg
+    ws, nws = r.workspace(b, QSA_OP_SPARSE_ATTN_DECODE, 0)
 
     def one():
-        d.q.copy_(hq, non_blocking=True)
-        d.idx_q.copy_(hiq, non_blocking=True)
-        d.idx_w.copy_(hiw, non_blocking=True)
-        d.idx_k_new.copy_(hik, non_blocking=True)
-        for i, (p, s) in enumerate(kv_dst):
-            d.k_pool[p, s].copy_(hk[i], non_blocking=True)
-            d.v_pool[p, s].copy_(hv[i], non_blocking=True)
-        w.step(True)
+        st.h2d(0)
+        d.k_pool[pages, slots] = st.view(0, "k")
+        d.v_pool[pages, slots] = st.view(0, "v")
+        r.compress(b, st.view(0, "idx_k"), d.new_seq, d.new_pos, d.kcomp_pool)
+        r.select(b, st.view(0, "idx_q"), st.view(0, "idx_w"), d.kcomp_pool, w.sel, w.n_sel)
+        qsa_sparse_attn_decode(cfg, b, st.view(0, "q"), d.k_pool, d.v_pool, w.sel, w.n_sel, w.out,
+                               None, 0, ws, nws)
         hout.copy_(w.out, non_blocking=True)
 
     for _ in range(warmup):
         one()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(steps):
         one()
-    b.record()
+    e.record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) * 1000 / steps, h2d, d2h
+    us = a.elapsed_time(e) * 1000 / steps
+    w.step(True)
+    torch.cuda.synchronize()
+    if not torch.equal(hout.view(torch.int16), w.out.cpu().view(torch.int16)):
+        raise RuntimeError("end-to-end decode output differs from the device step's output")
+    return us, st.nbytes, hout.numel() * hout.element_size()
 
 
 def dense_time_ms(w: Workload, decode: bool, reps: int, flush=None):
@@ -543,7 +598,7 @@ def main():
                     + work["attn_bytes"] / (peaks["hbm"] * 1e9)) * 1e3
     log(f"prefill {c.name}: {ms_step:.3f} ms/step, {value / 1e6:.3f} M tok/s, stages "
         + ", ".join(f"{k} {v['ms']:.3f} ms ({100 * v['frac']:.1f}% {v['bound']})" for k, v in stages.items()))
-    e2e_ms, h2d, d2h = e2e_prefill(w, max(3, args.steps // 3), 2)
+    e2e_ms, h2d, d2h = e2e_prefill(w, max(3, args.steps), 2)
     e2e_ms = max_over_ranks(e2e_ms, dist)
     log(f"prefill e2e {e2e_ms:.3f} ms/step")
     dense_ms = dense_time_ms(w, False, 1)
