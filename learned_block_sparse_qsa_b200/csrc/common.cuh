@@ -141,11 +141,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
-// L2 prefetch of a global range (no completion to track); bytes a multiple of 16.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
-}
-
 // ---------------------------------------------------------------- ordering keys
 // Monotone map of fp32 onto uint32 (larger float -> larger integer); -0 is folded onto +0 by
 // the caller so that equal scores compare equal.
@@ -170,11 +165,6 @@ __device__ __forceinline__ float key_score(unsigned long long k) {
   return ordered_to_f32((uint32_t)(k >> 32));
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 __device__ __forceinline__ int warp_sum_i(int v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
