@@ -124,3 +124,20 @@ def test_split_lists_many_rows_warp_lists():
     run = Run(c, integer=True, score_path=3).step()
     check_rows(run, range(c.num_q), True)
     assert run.runner.error_bits() == 0
+
+
+@pytest.mark.parametrize("positions", [1, 2, 8])
+def test_multi_token_decode_widths(positions):
+    """1 to 8 query positions per sequence (multi-token-prediction verify widths): row tiles of
+    four hold one sequence's rows, parts of two sequences, or one sequence over two tiles."""
+    c = Config(f"dec_b3x{positions}_ctx65536", "decode", 3, 65536, positions, 32, 4, 128, 4, 128,
+               needles=4, shuffle_pages=True, seed=0xDEC4 + positions)
+    run = Run(c, integer=True, score_path=3).step(compress=positions % 4 == 0)
+    o = check_rows(run, range(c.num_q), True)
+    h = host(c, True)
+    q_seq, q_pos = h.rows()
+    for r in sorted({0, c.num_q - 1}):
+        t, n = int(q_pos[r]), o["n_sel"][r]
+        ref_o, ref_lse = orc.attend(h.q([r])[0], *h.kv(int(q_seq[r]), orc.expand(o["sel"][r][:n], t)))
+        check_attention(o["out"][r], o["lse"][r], ref_o, ref_lse)
+    assert run.runner.error_bits() == 0
