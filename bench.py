@@ -381,7 +381,8 @@ def e2e_prefill(w: Workload, steps: int, warmup: int):
 def e2e_decode(w: Workload, steps: int, warmup: int):
     """Whole decode step through the public API with host inputs: one host-to-device copy of the
     step's inputs (queries, indexer tensors, the new tokens' K/V rows), the rows scattered into the
-    cache, the layer, one device-to-host copy of the output every step."""
+    cache, the layer, one device-to-host copy of the output every step; the step is captured once
+    as a CUDA graph and replayed."""
     torch = w.torch
     c, d = w.c, w.di
     q_pos = d.q_pos.long()
@@ -407,17 +408,32 @@ def e2e_decode(w: Workload, steps: int, warmup: int):
                                None, 0, ws, nws)
         hout.copy_(w.out, non_blocking=True)
 
-    for _ in range(warmup):
+    # the whole step -- copy in, scatter, the layer's calls, copy out -- as one CUDA graph, the
+    # way a serving loop replays it
+    for _ in range(max(warmup, 1)):
         one()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        one()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        one()
+    for _ in range(warmup):
+        g.replay()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(steps):
-        one()
+        g.replay()
     e.record()
     torch.cuda.synchronize()
     us = a.elapsed_time(e) * 1000 / steps
+    del g
     w.step(True)
     torch.cuda.synchronize()
     if not torch.equal(hout.view(torch.int16), w.out.cpu().view(torch.int16)):

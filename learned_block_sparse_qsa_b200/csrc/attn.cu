@@ -374,7 +374,7 @@ struct SwCfg {
   static constexpr int ROW_OFF = POS_OFF + NST * NBS * 4 * 4;
   static constexpr int BLK_OFF = ROW_OFF + kMaxSel * 4;
   static constexpr int BAR_OFF = BLK_OFF + kMaxSel * 4;
-  static constexpr int TOTAL = BAR_OFF + 2 * NST * 8 + 16;
+  static constexpr int TOTAL = BAR_OFF + (2 * NST + 1) * 8 + 8;  // full, empty, combine barriers
   static constexpr int THREADS = (NCW + 1) * 32;
   static_assert(NBS <= 32, "one producer lane per block slot");
 };
@@ -392,6 +392,7 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
   int* sBlk = reinterpret_cast<int*>(smem + C::BLK_OFF);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + C::NST;
+  uint64_t* cbar = empty + C::NST;  // split-K combine: the row's partials arriving
   const uint32_t sbase = smem_addr(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row = blockIdx.x, split = blockIdx.y;
@@ -415,6 +416,7 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], C::NCW);
     }
+    mbar_init(cbar, 1);
     mbar_fence_init();
   }
   {  // every thread: one round of (selection entry -> page table) loads for the CTA's slice
@@ -601,40 +603,52 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
     sL[2 * qc + 1] = l1;
   }
   asm volatile("bar.sync 1, %0;\n" ::"n"(C::NCW * 32));
-  // one warp per (KV head gg, query head h of its group), lanes across the head dims
-  const int lg = __ffs(G) - 1;  // G is a power of two
-  for (int c = warp; c < HKV * G; c += C::NCW) {
-    const int gg = c >> lg, h = c & (G - 1);
-    float f[C::NSLC];
-    float M = -INFINITY, L = 0.f;
+  // every consumer thread merges 4 head dims of one query head at a time: the slices' m and l
+  // give the weights, then one 16-byte read per slice and one 8- or 16-byte store
+  {
+    constexpr int D4 = D / 4;
+    const int lg = __ffs(G) - 1;  // G is a power of two
+    const int n4 = HKV * G * D4;
+    const float* sm = reinterpret_cast<const float*>(smem);
+#pragma unroll 4
+    for (int e = tid; e < n4; e += C::NCW * 32) {
+      const int hq = e / D4, d = (e % D4) * 4;
+      const int gg = hq >> lg, h = hq & (G - 1);
+      float ms[C::NSLC], f[C::NSLC];
+      float M = -INFINITY, L = 0.f;
 #pragma unroll
-    for (int sl = 0; sl < C::NSLC; ++sl)
-      M = fmaxf(M, (reinterpret_cast<float*>(smem) + (sl * HKV + gg) * (8 * D + 16))[8 * D + h]);
+      for (int sl = 0; sl < C::NSLC; ++sl) {
+        ms[sl] = sm[(sl * HKV + gg) * (8 * D + 16) + 8 * D + h];
+        M = fmaxf(M, ms[sl]);
+      }
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int sl = 0; sl < C::NSLC; ++sl) {
-      const float* base = reinterpret_cast<float*>(smem) + (sl * HKV + gg) * (8 * D + 16);
-      const float ms = base[8 * D + h];
-      f[sl] = (M != -INFINITY && ms != -INFINITY) ? exp2f(ms - M) : 0.f;
-      L += base[8 * D + 8 + h] * f[sl];
-    }
-    const int hq = gg * G + h;
-    const float inv = L > 0.f ? 1.0f / L : 0.f;
-    const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
-    const long long pi = ((long long)row * a.splits + split) * a.Hq + hq;
-    for (int d = lane; d < D; d += 32) {
-      float O = 0.f;
-#pragma unroll
-      for (int sl = 0; sl < C::NSLC; ++sl)
-        O += (reinterpret_cast<float*>(smem) + (sl * HKV + gg) * (8 * D + 16))[h * D + d] * f[sl];
-      const float res = O * inv;
-      if (a.splits == 1) a.out[((long long)row * a.Hq + hq) * D + d] = __float2bfloat16_rn(res);
-      else a.part_o[pi * D + d] = res;
-    }
-    if (lane == 0) {
+      for (int sl = 0; sl < C::NSLC; ++sl) {
+        const float* base = sm + (sl * HKV + gg) * (8 * D + 16);
+        f[sl] = (M != -INFINITY && ms[sl] != -INFINITY) ? exp2f(ms[sl] - M) : 0.f;
+        L += base[8 * D + 8 + h] * f[sl];
+        const float4 o = *reinterpret_cast<const float4*>(base + h * D + d);
+        O.x = fmaf(o.x, f[sl], O.x);
+        O.y = fmaf(o.y, f[sl], O.y);
+        O.z = fmaf(o.z, f[sl], O.z);
+        O.w = fmaf(o.w, f[sl], O.w);
+      }
+      const float inv = L > 0.f ? 1.0f / L : 0.f;
+      const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
+      O.x *= inv;
+      O.y *= inv;
+      O.z *= inv;
+      O.w *= inv;
       if (a.splits == 1) {
-        if (a.lse) a.lse[(long long)row * a.Hq + hq] = lse2 * 0.69314718055994531f;
+        uint2 packed;
+        packed.x = pack_bf16(O.x, O.y);
+        packed.y = pack_bf16(O.z, O.w);
+        *reinterpret_cast<uint2*>(a.out + ((long long)row * a.Hq + hq) * D + d) = packed;
+        if (d == 0 && a.lse) a.lse[(long long)row * a.Hq + hq] = lse2 * 0.69314718055994531f;
       } else {
-        a.part_lse[pi] = lse2;
+        const long long pi = ((long long)row * a.splits + split) * a.Hq + hq;
+        *reinterpret_cast<float4*>(a.part_o + pi * D + d) = O;
+        if (d == 0) a.part_lse[pi] = lse2;
       }
     }
   }
@@ -651,9 +665,23 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
       __threadfence();
       const int S = a.splits, Hq = a.Hq;
       const long long b0 = (long long)row * S * Hq;  // partial index of (split 0, head 0)
+      const int nv = Hq * D / 4;                      // float4 groups of one split's output
+      // the row's partials are contiguous ([S][Hq][D] fp32): when they fit in the idle stage
+      // ring, bulk copies bring them in while the weights below are computed
+      const uint32_t pbytes = (uint32_t)S * Hq * D * 4;
+      const bool staged = (size_t)pbytes + (size_t)Hq * S * 4 <= (size_t)C::BIG;
+      if (staged && tid == 0) {
+        // generic-proxy partials of the other splits (ordered by their fences and the counter),
+        // and this CTA's earlier shared-memory use, before the async-proxy copies
+        asm volatile("fence.proxy.async;\n" ::: "memory");
+        mbar_arrive_expect_tx(cbar, pbytes);
+        const uint32_t per = (uint32_t)Hq * D * 4;
+        for (int sp = 0; sp < S; ++sp)
+          bulk_g2s(sbase + sp * per, a.part_o + (b0 + (long long)sp * Hq) * D, per, cbar);
+      }
       // weights 2^(lse_s - M) / sum into shared memory [Hq][S]: every (head, split) log-sum-exp
       // is loaded at once, then one thread per head reduces its S values
-      float* wn = reinterpret_cast<float*>(smem);
+      float* wn = reinterpret_cast<float*>(smem + (staged ? pbytes : 0u));
       for (int p = tid; p < Hq * S; p += C::THREADS) {
         const int hq = p / S, sp = p % S;
         wn[p] = __ldcg(a.part_lse + b0 + (long long)sp * Hq + hq);
@@ -674,43 +702,64 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
           a.lse[(long long)row * Hq + tid] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
       }
       __syncthreads();
-      // outputs: each thread owns up to 4 float4 groups of head dims and walks the splits once,
-      // so that 4 independent 16-byte loads per split (12 with the unrolling) are in flight
-      constexpr int VPT = 4;
-      const long long sstride = (long long)Hq * D / 4;  // float4s between splits
-      const float4* part4 = reinterpret_cast<const float4*>(a.part_o) + b0 * D / 4;
-      const int nv = Hq * D / 4;
-      for (int v0 = tid; v0 < nv; v0 += VPT * C::THREADS) {
-        float4 acc[VPT];
-        int hqv[VPT];
-#pragma unroll
-        for (int j = 0; j < VPT; ++j) {
-          acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-          hqv[j] = (v0 + j * C::THREADS) * 4 / D;
+      bf16* orow = a.out + (long long)row * Hq * D;
+      if (staged) {
+        if (mbar_wait(cbar, 0, a.err)) {
+          const float4* ps = reinterpret_cast<const float4*>(smem);
+          for (int v = tid; v < nv; v += C::THREADS) {
+            const float* w = wn + (v * 4 / D) * S;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int sp = 0; sp < S; ++sp) {
+              const float4 p = ps[sp * nv + v];
+              acc.x = fmaf(w[sp], p.x, acc.x);
+              acc.y = fmaf(w[sp], p.y, acc.y);
+              acc.z = fmaf(w[sp], p.z, acc.z);
+              acc.w = fmaf(w[sp], p.w, acc.w);
+            }
+            uint2 packed;
+            packed.x = pack_bf16(acc.x, acc.y);
+            packed.y = pack_bf16(acc.z, acc.w);
+            *reinterpret_cast<uint2*>(orow + (long long)v * 4) = packed;
+          }
         }
+      } else {
+        // outputs: each thread owns up to 4 float4 groups of head dims and walks the splits
+        // once, so that 4 independent 16-byte loads per split (12 with the unrolling) are in flight
+        constexpr int VPT = 4;
+        const long long sstride = (long long)Hq * D / 4;  // float4s between splits
+        const float4* part4 = reinterpret_cast<const float4*>(a.part_o) + b0 * D / 4;
+        for (int v0 = tid; v0 < nv; v0 += VPT * C::THREADS) {
+          float4 acc[VPT];
+          int hqv[VPT];
+#pragma unroll
+          for (int j = 0; j < VPT; ++j) {
+            acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            hqv[j] = (v0 + j * C::THREADS) * 4 / D;
+          }
 #pragma unroll 3
-        for (int sp = 0; sp < S; ++sp) {
+          for (int sp = 0; sp < S; ++sp) {
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) {
+              const int v = v0 + j * C::THREADS;
+              if (v < nv) {
+                const float w = wn[hqv[j] * S + sp];
+                const float4 p = __ldcg(part4 + sp * sstride + v);
+                acc[j].x = fmaf(w, p.x, acc[j].x);
+                acc[j].y = fmaf(w, p.y, acc[j].y);
+                acc[j].z = fmaf(w, p.z, acc[j].z);
+                acc[j].w = fmaf(w, p.w, acc[j].w);
+              }
+            }
+          }
 #pragma unroll
           for (int j = 0; j < VPT; ++j) {
             const int v = v0 + j * C::THREADS;
             if (v < nv) {
-              const float w = wn[hqv[j] * S + sp];
-              const float4 p = __ldcg(part4 + sp * sstride + v);
-              acc[j].x = fmaf(w, p.x, acc[j].x);
-              acc[j].y = fmaf(w, p.y, acc[j].y);
-              acc[j].z = fmaf(w, p.z, acc[j].z);
-              acc[j].w = fmaf(w, p.w, acc[j].w);
+              uint2 packed;
+              packed.x = pack_bf16(acc[j].x, acc[j].y);
+              packed.y = pack_bf16(acc[j].z, acc[j].w);
+              *reinterpret_cast<uint2*>(orow + (long long)v * 4) = packed;
             }
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < VPT; ++j) {
-          const int v = v0 + j * C::THREADS;
-          if (v < nv) {
-            uint2 packed;
-            packed.x = pack_bf16(acc[j].x, acc[j].y);
-            packed.y = pack_bf16(acc[j].z, acc[j].w);
-            *reinterpret_cast<uint2*>(a.out + (long long)row * Hq * D + (long long)v * 4) = packed;
           }
         }
       }

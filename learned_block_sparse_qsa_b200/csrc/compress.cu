@@ -25,6 +25,11 @@ __global__ void __launch_bounds__(256) compress_kernel(
   const int ch = (int)(tid % CH);
   if (grp >= n_groups) return;
   const long long r0 = grp * 4;
+  // the four raw keys do not depend on the checks below: their loads go out first, so that
+  // only the page-table read waits on the row metadata
+  uint4 raw[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) raw[i] = __ldg(reinterpret_cast<const uint4*>(idx_k + (r0 + i) * DI) + ch);
   const int seq = new_seq[r0];
   const int pos0 = new_pos[r0];
   bool ok = (pos0 >= 0) && (pos0 % 4 == 0);
@@ -53,8 +58,7 @@ __global__ void __launch_bounds__(256) compress_kernel(
   for (int e = 0; e < 8; ++e) acc[e] = 0.0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(idx_k + (r0 + i) * DI) + ch);
-    const bf16* h = reinterpret_cast<const bf16*>(&v);
+    const bf16* h = reinterpret_cast<const bf16*>(&raw[i]);
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] += (double)__bfloat162float(h[e]);
   }

@@ -107,6 +107,22 @@ __device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* m, int x,
       "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_addr(bar))
       : "memory");
 }
+// The same load with an L2 eviction-priority policy (from l2_evict_first_policy below).
+__device__ __forceinline__ void tma2d_hint(uint32_t dst, const CUtensorMap* m, int x, int y, uint64_t* bar,
+                                           uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(dst),
+      "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+// Lines read once per call: first in line for eviction, so that the small tables read next
+// (page table, selections) stay in L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
 __device__ __forceinline__ void tma3d(uint32_t dst, const CUtensorMap* m, int x, int y, int z, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),

@@ -277,8 +277,9 @@ __global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
         // the stage's earlier ldmatrix reads (generic proxy) before the TMA writes (async proxy)
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         mbar_arrive_expect_tx(&bar[s], DS_PAGE);
-        tma2d(stage0 + s * DS_PAGE, &tmK, 0, pg * 16, &bar[s]);
-        tma2d(stage0 + s * DS_PAGE + DS_PAGE / 2, &tmK, 64, pg * 16, &bar[s]);
+        const uint64_t pol = l2_evict_first_policy();
+        tma2d_hint(stage0 + s * DS_PAGE, &tmK, 0, pg * 16, &bar[s], pol);
+        tma2d_hint(stage0 + s * DS_PAGE + DS_PAGE / 2, &tmK, 64, pg * 16, &bar[s], pol);
       } else {
         mbar_arrive(&bar[s]);  // no data: the page's blocks are masked below
       }
@@ -662,15 +663,20 @@ __global__ void __launch_bounds__(DM_THREADS)
     redn[warp] = nk;
   }
   __syncthreads();
-  nk = 0;
-  lo = ~0ull;
-  hi = 0ull;
-  mb = 0ull;
-  for (int w = 0; w < NW; ++w) {
-    nk += redn[w];
-    lo = red[w] < lo ? red[w] : lo;
-    hi = red[16 + w] > hi ? red[16 + w] : hi;
-    mb = red[32 + w] > mb ? red[32 + w] : mb;
+  // every warp reduces the NW per-warp entries itself: one entry per lane, then shuffles
+  static_assert(NW <= 32, "one per-warp entry per lane");
+  nk = lane < NW ? redn[lane] : 0u;
+  lo = lane < NW ? red[lane] : ~0ull;
+  hi = lane < NW ? red[16 + lane] : 0ull;
+  mb = lane < NW ? red[32 + lane] : 0ull;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    nk += __shfl_xor_sync(0xffffffffu, nk, o);
+    const u64 x = __shfl_xor_sync(0xffffffffu, lo, o), y = __shfl_xor_sync(0xffffffffu, hi, o),
+              z = __shfl_xor_sync(0xffffffffu, mb, o);
+    lo = x < lo ? x : lo;
+    hi = y > hi ? y : hi;
+    mb = z > mb ? z : mb;
   }
   if ((int)nk < need) {  // lists dropped too much: the exact kernel redoes the row
     if (tid == 0) ws.redo[row] = 1;
