@@ -24,6 +24,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -147,8 +148,17 @@ def traffic_for(kernel_file: str, key: str):
     if not d:
         return None
     src = os.path.join(ROOT, "learned_block_sparse_qsa_b200", "csrc", kernel_file)
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return d["bytes_per_launch"] if d.get("source_sha") == h else None
+    return d["bytes_per_launch"] if d.get("source_sha") == code_sha(src) else None
+
+
+def code_sha(path: str) -> str:
+    """Hash of a CUDA source with comments and blank space removed: counters stay attached to
+    the code they were taken on, and an edit of a comment does not orphan them."""
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = " ".join(text.split())
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
 
 
 # ------------------------------------------------------------------------------------ workload

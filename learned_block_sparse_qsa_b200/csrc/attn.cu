@@ -8,16 +8,24 @@
 //
 // B200 design.  The work is a gather: per query token up to 513 blocks x 4 positions x Hkv x D x
 // 2 (K,V) x 2 bytes = 4.2 MB at Hkv = 4, D = 128, for 8 flop/byte -- HBM-bound, far from the tensor
-// roofline.  One CTA serves one query row (or one split of it):
-//  * a producer warp turns selection entries into physical rows (page table, causal clip at t)
-//    and issues one 1-D bulk copy (TMA engine, cp.async.bulk) per position row of K and of V
-//    (Hkv*D*2 = 1 KiB each) into a 3-stage ring of shared memory, completion on an mbarrier;
-//    rows are stored with a 16-byte skew per row, so the ldmatrix reads below are conflict-free;
-//  * 8 consumer warps: warp (g, slice) takes KV head g and every NSLC-th 16-position chunk; the
-//    8 (or fewer) query heads of group g are the M=16 rows of mma.m16n8k16 (padding rows are
-//    zero), positions are N; online softmax in fp32 (exp2 domain), P in bf16 into P*V;
-//  * slices of one head group are merged through shared memory at the end; split-K partials
-//    (decode) go to the workspace and a combine kernel merges them by log-sum-exp.
+// roofline.  One CTA serves one query row (or one split of it).
+//
+// sparse_attn_sw_kernel (Hq/Hkv <= 8, every configuration measured here):
+//  * all threads first turn the CTA's selection entries into physical rows (page table, causal
+//    clip at t); a producer warp then issues one 4 KB bulk copy (TMA engine, cp.async.bulk) per
+//    selected block of K and of V -- a block's 4 positions x all KV heads are contiguous in a
+//    page -- into a 3-stage ring, with block slots skewed by 16 bytes so that ldmatrix is
+//    conflict-free;
+//  * consumer warp (g, slice) takes KV head g and every NSLC-th group of 4 blocks; the MMAs run
+//    swap-AB: positions are the M = 16 rows of mma.m16n8k16 and the group's query heads are N = 8,
+//    so no MMA row is padding; online softmax in fp32 (exp2 domain), P in bf16 into P*V;
+//  * the slices of each KV head merge through shared memory, every consumer thread taking 4 head
+//    dims of one query head; split-K partials (decode) go to the workspace, and the last split of
+//    the row to finish (a per-row counter) bulk-copies them into its idle stage ring and merges
+//    them by log-sum-exp.
+//
+// sparse_attn_kernel (Hq/Hkv > 8): one bulk copy per position row (Hkv x D x 2 bytes), the query
+// heads of a group as the MMA rows, and split-K partials merged by combine_kernel.
 #include "common.cuh"
 #include "internal.h"
 
