@@ -1,6 +1,7 @@
 """Host logic of bench.py that needs no GPU: the source hash that keeps committed ncu traffic
 figures attached to the kernel code they were measured on."""
 
+
 def test_code_sha_ignores_comments_but_not_code(tmp_path):
     import bench
 
