@@ -54,6 +54,14 @@ struct AttnArgs {
 };
 
 
+// The producer warp leaves only after the last (up to nst) stages it posted have landed: in the
+// normal course they already have, and after a wait that ran out (already flagged) this is the
+// bounded wait for the bulk copies still in flight into this CTA's shared memory.
+__device__ __forceinline__ void drain_stages(uint64_t* full, int posted, int nst, int lane, int32_t* err) {
+  if (lane != 0) return;
+  for (int j = posted > nst ? posted - nst : 0; j < posted; ++j) mbar_wait(&full[j % nst], (j / nst) & 1, err);
+}
+
 template <int D, int HKV>
 struct AttnCfg {
   static constexpr int NCW = 8;                // consumer warps
@@ -116,7 +124,8 @@ __global__ void __launch_bounds__(AttnCfg<D, HKV>::THREADS, 1) sparse_attn_kerne
     constexpr int RPL = (C::ROWS + 31) / 32;  // rows per lane
     const int32_t* selrow = a.sel + (long long)row * a.sel_stride;
     const int32_t* ptab = a.page_table + (long long)(ok ? seq : 0) * a.max_pages;
-    for (int it = 0; it < nstages; ++it) {
+    int it = 0;
+    for (; it < nstages; ++it) {
       const int st = it % C::NST;
       if (it >= C::NST && !mbar_wait(&empty[st], ((it / C::NST) - 1) & 1, a.err)) break;
       const uint32_t kdst = sbase + st * C::STAGE;
@@ -176,6 +185,7 @@ __global__ void __launch_bounds__(AttnCfg<D, HKV>::THREADS, 1) sparse_attn_kerne
         }
       }
     }
+    drain_stages(full, it, C::NST, lane, a.err);
     return;
   }
 
@@ -448,7 +458,8 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
 
   if (warp == C::NCW) {
     // ================================================================ producer
-    for (int it = 0; it < nstages; ++it) {
+    int it = 0;
+    for (; it < nstages; ++it) {
       const int st = it % C::NST;
       if (it >= C::NST && !mbar_wait(&empty[st], ((it / C::NST) - 1) & 1, a.err)) break;
       const uint32_t kdst = sbase + st * C::STAGE + lane * C::BPITCH;
@@ -496,6 +507,7 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
         }
       }
     }
+    drain_stages(full, it, C::NST, lane, a.err);
   } else {
   // ================================================================== consumers
   const int g = warp % HKV;
@@ -712,7 +724,9 @@ __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw
       __syncthreads();
       bf16* orow = a.out + (long long)row * Hq * D;
       if (staged) {
-        if (mbar_wait(cbar, 0, a.err)) {
+        if (!mbar_wait(cbar, 0, a.err)) {
+          mbar_wait(cbar, 0, a.err);  // ran out: wait once more, bounded, for the copies in flight
+        } else {
           const float4* ps = reinterpret_cast<const float4*>(smem);
           for (int v = tid; v < nv; v += C::THREADS) {
             const float* w = wn + (v * 4 / D) * S;

@@ -630,7 +630,10 @@ __global__ void __launch_bounds__(DM_THREADS)
   }
   const bool arrived = mbar_wait(bar, 0, a.err);
   if (!__syncthreads_and(arrived)) {  // reported as a timeout; the exact kernel redoes the row
-    if (tid == 0) ws.redo[row] = 1;
+    if (tid == 0) {
+      ws.redo[row] = 1;
+      mbar_wait(bar, 0, a.err);  // and the copies still in flight land first (bounded)
+    }
     return;
   }
 
