@@ -9,6 +9,8 @@
 // TQ consecutive tokens of one sequence), streams the sequence's pages (64 positions) of that KV
 // head through a 3-stage cp.async ring, and keeps fp32 online-softmax state in registers.  The
 // decode form splits the context across CTAs and merges by log-sum-exp.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -282,13 +284,40 @@ cudaError_t run_dense(const DenseArgs& a, int splits, cudaStream_t s) {
 
 }  // namespace
 
+namespace {
+// CTAs of the kernel instance that one SM holds at once (its shared memory decides), looked up
+// once per process; 1 when the runtime cannot say (no device), with the error cleared.
+template <int D, int MR>
+int dense_resident_ctas() {
+  static std::atomic<int> cached{0};
+  const int c = cached.load(std::memory_order_relaxed);
+  if (c > 0) return c;
+  using C = DenseCfg<D, MR>;
+  int n = 0;
+  if (set_smem_once(dense_attn_kernel<D, MR>, C::TOTAL) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dense_attn_kernel<D, MR>, C::THREADS, C::TOTAL) !=
+          cudaSuccess ||
+      n < 1) {
+    cudaGetLastError();
+    return 1;
+  }
+  cached.store(n, std::memory_order_relaxed);
+  return n;
+}
+}  // namespace
+
+// Automatic split count: as many splits as fill the GPU in ONE wave of resident CTAs (a second,
+// nearly empty wave would double the time of the whole launch), capped at one page per split.
 int resolve_dense_splits(const Geometry& g, int requested) {
   if (requested > 0) return requested;
-  const int mr = g.num_q <= 256 ? 32 : 64;
+  const bool small = g.num_q <= 256;
+  const int mr = small ? 32 : 64;
   const int tq = mr / g.G;
   const int tiles = (g.num_q + tq - 1) / tq;
   const int ctas = tiles * g.Hkv;
-  int s = (2 * num_sms() + ctas - 1) / ctas;
+  const int per_sm = g.D == 64 ? (small ? dense_resident_ctas<64, 32>() : dense_resident_ctas<64, 64>())
+                               : (small ? dense_resident_ctas<128, 32>() : dense_resident_ctas<128, 64>());
+  int s = per_sm * num_sms() / ctas;
   const int pages = g.max_pos / 64 + 1;
   if (s > pages) s = pages;
   if (s < 1) s = 1;
