@@ -166,3 +166,65 @@ def test_short_rows_keep_every_candidate():
     s = np.random.default_rng(3).standard_normal(300).astype(np.float32)
     got = model_select(s, 128)
     assert got is not None and np.array_equal(got, np.arange(300))
+
+
+# --------------------------------------------------------------------------------------------
+# The prefill indexer's sampled threshold.  The tile sequence is first every 32nd tile of 128
+# blocks (the sample), then all tiles.  Each half-row (blocks 64h..64h+63 of every tile) keeps its
+# 32 best sampled scores.  The row threshold is the smaller of the two halves' 32nd best (minus
+# infinity when the row has no more candidates than the budget, or a half sampled fewer than 32).
+# Every key at or above it is kept, and the exact select runs over the kept keys.  The row is
+# handed to the exact path when fewer than need keys were kept, or a half-row kept more than its
+# 2,048 slots.
+
+TILE, SAMPLE_EVERY, SAMPLE_KEEP, HALF_CAP = 128, 32, 32, 2048
+
+
+def sampled_select(scores32: np.ndarray, topk: int = 512):
+    n = scores32.shape[0]
+    need = min(topk, n)
+    keys = make_keys(scores32)
+    blocks = np.arange(n)
+    half = (blocks % TILE) // (TILE // 2)
+    sampled = (blocks // TILE) % SAMPLE_EVERY == 0
+    if n <= topk:
+        tau_key = np.uint64(0)
+    else:
+        taus = []
+        for h in (0, 1):
+            s = np.sort(keys[sampled & (half == h)])[::-1]
+            taus.append(int(s[SAMPLE_KEEP - 1]) >> 32 if s.shape[0] >= SAMPLE_KEEP else 0)
+        tau_key = np.uint64(min(taus) << 32)  # a score threshold: every block at that score
+    kept = keys[keys >= tau_key]
+    if kept.shape[0] < need or any(np.sum((keys >= tau_key) & (half == h)) > HALF_CAP for h in (0, 1)):
+        return None
+    top = np.sort(kept)[::-1][:need]
+    return np.sort((np.uint64(0xFFFFFFFF) - (top & np.uint64(0xFFFFFFFF))).astype(np.int64))
+
+
+@pytest.mark.parametrize("n,seed", [(262144, 0), (262144, 1), (32768, 2), (32768, 3)])
+def test_sampled_threshold_is_exact_without_redo_at_chunk_scale(n, seed):
+    """Rows of the C4 and C2 prefill chunks (about 262,144 and 32,768 candidates)."""
+    s = np.random.default_rng(seed).standard_normal(n).astype(np.float32)
+    got = sampled_select(s)
+    assert got is not None
+    assert np.array_equal(got, oracle_select(s))
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_sampled_threshold_kept_rows_are_exact(seed):
+    s, _, topk = mixed_case(seed)
+    got = sampled_select(s, topk)
+    if got is not None:
+        assert np.array_equal(got, oracle_select(s, topk))
+
+
+def test_sampled_threshold_hands_over_rows_just_above_the_budget():
+    """Just above 512 candidates the sample is one tile, whose 32nd best per half keeps about
+    half of the row: fewer than 512 keys, so the exact path takes it. This is a cost, not an
+    error; long rows keep about 2,048."""
+    s = np.random.default_rng(5).standard_normal(700).astype(np.float32)
+    assert sampled_select(s) is None
+    s = np.random.default_rng(6).standard_normal(3000).astype(np.float32)
+    got = sampled_select(s)
+    assert got is not None and np.array_equal(got, oracle_select(s))
