@@ -395,7 +395,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       // -- row threshold: every epilogue warp arrives here once per segment with tiles
       if (L > 0) {
-        m->thr[hf][row] = (lim > a.topk) ? mn : -INFINITY;
+        // a row of at most 2 * TC_CAP candidates keeps every key (each half-row holds at most
+        // TC_CAP): a sample of one or two tiles would keep too few of them for the exact select
+        m->thr[hf][row] = (lim > a.topk && lim > 2 * TC_CAP) ? mn : -INFINITY;
         epi_sync();
         tau = fminf(m->thr[0][row], m->thr[1][row]);
       }

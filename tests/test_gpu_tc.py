@@ -61,10 +61,12 @@ def test_tc_small_budget_exact():
     check_rows(run, range(0, 3000, 7), True, topk=37)
 
 
-def test_tc_fallback_on_decreasing_scores():
-    """Scores that fall with the block index defeat the sampled threshold (the sample's best blocks
-    are the first ones), so rows go to the exact fallback -- the result must still be exact."""
-    c = TC_PREFILL.replace(ctx=4096, n_new=4096)
+@pytest.mark.parametrize("ctx,n_new", [(4096, 4096), (32768, 2048)], ids=["short_rows", "sampled_rows"])
+def test_tc_fallback_on_decreasing_scores(ctx, n_new):
+    """Scores that fall with the block index: rows of up to 4,096 candidates keep every key and
+    need no fallback; longer rows defeat the sampled threshold (the sample's best blocks are the
+    first ones) and go to the exact fallback.  Both must be exact."""
+    c = TC_PREFILL.replace(ctx=ctx, n_new=n_new)
     run = Run(c, integer=True, score_path=1)
     nb = c.ctx // 4
     vals = np.zeros((c.ctx, c.Di), dtype=np.float32)
@@ -73,7 +75,10 @@ def test_tc_fallback_on_decreasing_scores():
     vals[:, 1] = (nb - blk) % 256
     kbits = torch.tensor(vals).to(torch.bfloat16)
     run.di.idx_k[0] = kbits.cuda()
-    run.di.idx_k_new.copy_(run.di.idx_k[0])
+    run.di.idx_k_new.copy_(run.di.idx_k[0, c.ctx_start:])
+    if c.ctx_start > 0:  # the prefix's compressed keys, from the keys planted above
+        run.di.kcomp_pool.zero_()
+        run.setup_prefix()
     q = np.zeros((c.num_q, 4, c.Di), dtype=np.float32)
     q[:, :, 0] = 256
     q[:, :, 1] = 1

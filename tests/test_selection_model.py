@@ -172,7 +172,8 @@ def test_short_rows_keep_every_candidate():
 # The prefill indexer's sampled threshold.  The tile sequence is first every 32nd tile of 128
 # blocks (the sample), then all tiles.  Each half-row (blocks 64h..64h+63 of every tile) keeps its
 # 32 best sampled scores.  The row threshold is the smaller of the two halves' 32nd best (minus
-# infinity when the row has no more candidates than the budget, or a half sampled fewer than 32).
+# infinity when the row has no more candidates than the budget or than the two half-row buffers
+# hold, or when a half sampled fewer than 32).
 # Every key at or above it is kept, and the exact select runs over the kept keys.  The row is
 # handed to the exact path when fewer than need keys were kept, or a half-row kept more than its
 # 2,048 slots.
@@ -187,7 +188,7 @@ def sampled_select(scores32: np.ndarray, topk: int = 512):
     blocks = np.arange(n)
     half = (blocks % TILE) // (TILE // 2)
     sampled = (blocks // TILE) % SAMPLE_EVERY == 0
-    if n <= topk:
+    if n <= topk or n <= 2 * HALF_CAP:
         tau_key = np.uint64(0)
     else:
         taus = []
@@ -219,12 +220,10 @@ def test_sampled_threshold_kept_rows_are_exact(seed):
         assert np.array_equal(got, oracle_select(s, topk))
 
 
-def test_sampled_threshold_hands_over_rows_just_above_the_budget():
-    """Just above 512 candidates the sample is one tile, whose 32nd best per half keeps about
-    half of the row: fewer than 512 keys, so the exact path takes it. This is a cost, not an
-    error; long rows keep about 2,048."""
-    s = np.random.default_rng(5).standard_normal(700).astype(np.float32)
-    assert sampled_select(s) is None
-    s = np.random.default_rng(6).standard_normal(3000).astype(np.float32)
-    got = sampled_select(s)
-    assert got is not None and np.array_equal(got, oracle_select(s))
+def test_sampled_threshold_keeps_every_key_of_rows_the_buffers_hold():
+    """Just above 512 candidates a one-tile sample would keep about half of the row (fewer than
+    512 keys, a redo); rows of up to 4,096 candidates keep every key instead, and are exact."""
+    for n, seed in ((700, 5), (1024, 6), (4096, 7), (6000, 8)):
+        s = np.random.default_rng(seed).standard_normal(n).astype(np.float32)
+        got = sampled_select(s)
+        assert got is not None and np.array_equal(got, oracle_select(s))
