@@ -21,7 +21,9 @@
 // Selection without in-loop compaction: the tile sequence is first every 32nd tile (a sample),
 // then all tiles.  During the sample each thread keeps the 32 best sampled scores of its half-row
 // in registers; the row threshold tau = min over its two halves of the 32nd best, so about 2,048
-// of the row's scores are >= tau, and fewer than 512 is a ~6-sigma event.  The full pass appends every (score >= tau, block) key to a
+// of the row's scores are >= tau, and fewer than 512 is a ~6-sigma event.  Rows of at most
+// 2 * TC_CAP candidates skip the threshold and keep every key (a sample of one or two tiles
+// would keep too few).  The full pass appends every (score >= tau, block) key to a
 // per-half-row buffer (in ascending block order); the final step checks that at least
 // min(512, t/4) keys were kept -- which proves every true top-512 key was kept -- and selects
 // exactly (radix select on 64-bit keys, lower block index wins ties) with a merge by rank.  Rows
