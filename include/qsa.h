@@ -84,8 +84,19 @@ typedef struct qsa_config {
   int32_t topk_blocks;  /* 1..512; the article's budget is 512 */
   int32_t page_tokens;  /* must be 64 */
   float softmax_scale;  /* <= 0 selects 1/sqrt(head_dim) */
-  int32_t score_path;   /* qsa_index_score_topk algorithm: 0 auto, 1 streaming, 2 materialised,
-                           3 split lists (idx_dim 128; falls back to 2 otherwise) */
+  int32_t score_path;   /* qsa_index_score_topk algorithm, every one exact and equal:
+                           0 auto: 3 for <= 128 rows when its plan fits, else 2 for <= 256 rows,
+                             else 1;
+                           1 many rows: at idx_dim 128 the tcgen05 tensor-core kernel, whose
+                             unsettled rows the streaming kernel redoes; else the streaming kernel;
+                           2 materialised scores (any shape);
+                           3 split lists for few rows (idx_dim 128; 2 when its plan does not fit);
+                           4 the mma.sync streaming kernel alone.
+                           Paths 1 and 3 at idx_dim 128 (and auto, which resolves to them) load
+                           operands through tensor maps: when the driver offers no tensor-map
+                           encoder, qsa_index_score_topk returns QSA_ERR_UNSUPPORTED rather than
+                           switch kernels silently.  The resolution itself depends on the shape
+                           only, so workspace sizes need no driver. */
 } qsa_config_t;
 
 typedef struct qsa_batch {
@@ -132,6 +143,16 @@ qsa_status_t qsa_index_score_topk(const qsa_config_t* cfg, const qsa_batch_t* ba
                                   const void* idx_q, const void* idx_w, const void* kcomp_pool,
                                   int32_t* sel, int32_t* n_sel, float* sel_scores,
                                   void* workspace, size_t ws_bytes, qsa_stream_t stream);
+
+/* Diagnostic, no counterpart in the article.  Paths 1 (idx_dim 128) and 3 first run a fast kernel
+ * that settles most rows and flags the rest, which the exact streaming kernel then recomputes.
+ * This host-only call returns in *flags the device address, inside `workspace`, of those flags
+ * (int32 [num_q]: 1 = the row was recomputed, 0 = the fast kernel's own result) as the last
+ * qsa_index_score_topk call with this config, batch shape and workspace left them; read them after
+ * that call has completed.  *flags = NULL when the resolved path keeps no flags (paths 2 and 4,
+ * path 1 below idx_dim 128, or an empty batch). */
+qsa_status_t qsa_index_score_redo_flags(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                        void* workspace, size_t ws_bytes, int32_t** flags);
 
 /* Diagnostic view of step (b): the fp32 score of every candidate block of every row, written to
  * scores (float [num_q, ld]); entries b >= t/4 are left untouched.  ld >= max_pos/4. */

@@ -79,6 +79,7 @@ _SIGS = {
     "qsa_index_compress": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p]),
     "qsa_index_score_topk": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qsa_index_score_redo_flags": (c_int32, [_S, _B, c_void_p, c_size_t, ctypes.POINTER(c_void_p)]),
     "qsa_index_scores": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
     "qsa_sparse_attn_prefill": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                           c_void_p, c_void_p, c_void_p]),
@@ -130,6 +131,15 @@ def qsa_index_score_topk(cfg, batch, idx_q, idx_w, kcomp_pool, sel, n_sel, sel_s
                                      _p(kcomp_pool), _p(sel), _p(n_sel), _p(sel_scores),
                                      _p(workspace), int(ws_bytes), _stream(stream)),
            "qsa_index_score_topk")
+
+
+def qsa_index_score_redo_flags(cfg, batch, workspace, ws_bytes) -> int | None:
+    """Device address of the redo flags (int32 [num_q]) inside the score workspace, or None."""
+    out = c_void_p(0)
+    _check(_lib.qsa_index_score_redo_flags(ctypes.byref(cfg), ctypes.byref(batch), _p(workspace),
+                                           int(ws_bytes), ctypes.byref(out)),
+           "qsa_index_score_redo_flags")
+    return out.value
 
 
 def qsa_index_scores(cfg, batch, idx_q, idx_w, kcomp_pool, scores, ld, stream=None):

@@ -49,7 +49,7 @@ qsa_status_t make_geometry(const qsa_config_t* cfg, const qsa_batch_t* b, Geomet
     return QSA_ERR_INVALID_ARG;
   if (!pow2_le(cfg->num_q_heads / cfg->num_kv_heads, 16)) return QSA_ERR_UNSUPPORTED;
   if (cfg->topk_blocks < 1 || cfg->topk_blocks > 512) return QSA_ERR_UNSUPPORTED;
-  if (cfg->score_path < 0 || cfg->score_path > 3) return QSA_ERR_INVALID_ARG;
+  if (cfg->score_path < 0 || cfg->score_path > 4) return QSA_ERR_INVALID_ARG;
   if ((long long)b->max_pages_per_seq * 64 > (1LL << 30)) return QSA_ERR_UNSUPPORTED;
   g->Hq = cfg->num_q_heads;
   g->Hkv = cfg->num_kv_heads;
@@ -143,8 +143,24 @@ qsa_status_t qsa_index_score_topk(const qsa_config_t* cfg, const qsa_batch_t* ba
   const size_t need = qsa::score_workspace_bytes(g, path);
   if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return QSA_ERR_WORKSPACE;
+  if (!qsa::score_path_runnable(g, path)) return QSA_ERR_UNSUPPORTED;
   return from_cuda(qsa::launch_score_topk(g, path, idx_q, idx_w, kcomp_pool, sel, n_sel,
                                           sel_scores, workspace, ws_bytes, (cudaStream_t)stream));
+}
+
+qsa_status_t qsa_index_score_redo_flags(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                        void* workspace, size_t ws_bytes, int32_t** flags) {
+  if (!flags) return QSA_ERR_INVALID_ARG;
+  *flags = nullptr;
+  Geometry g;
+  qsa_status_t st = make_geometry(cfg, batch, &g, false);
+  if (st != QSA_OK) return st;
+  const int path = qsa::resolve_score_path(g, cfg->score_path);
+  if (!workspace || ws_bytes < qsa::score_workspace_bytes(g, path)) return QSA_ERR_WORKSPACE;
+  size_t off = 0;
+  if (g.num_q > 0 && qsa::score_redo_offset(g, path, &off))
+    *flags = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + off);
+  return QSA_OK;
 }
 
 qsa_status_t qsa_index_scores(const qsa_config_t* cfg, const qsa_batch_t* batch,

@@ -25,6 +25,8 @@ cudaError_t launch_compress(const Geometry& g, const void* idx_k, const int32_t*
 // score.cu
 size_t score_workspace_bytes(const Geometry& g, int path);
 int resolve_score_path(const Geometry& g, int requested);
+bool score_path_runnable(const Geometry& g, int path);  // false: the driver lacks what it needs
+bool score_redo_offset(const Geometry& g, int path, size_t* off);
 cudaError_t launch_score_topk(const Geometry& g, int path, const void* idx_q, const void* idx_w,
                               const void* kcomp, int32_t* sel, int32_t* n_sel, float* sel_scores,
                               void* ws, size_t ws_bytes, cudaStream_t s);

@@ -13,7 +13,11 @@
 // cudaGetSymbolAddress and caches it.  That first call therefore makes a synchronous runtime call
 // and should come before any stream capture.  All calls share the array: calls that overlap on
 // the GPU (different streams, or different host threads) race on it.  Nothing in it has to start
-// at zero -- every partial the combine step reads is written earlier in the same call.
+// at zero -- every partial the combine step reads is written earlier in the same call.  The
+// per-device address cache itself is safe to fill from several host threads at once: each entry
+// is atomic, and threads that race on a device's first call store the same address.
+#include <atomic>
+
 #include "../../include/qsa.h"
 #include "internal.h"
 
@@ -22,7 +26,7 @@ namespace {
 constexpr size_t kScratchBytes = size_t(4) << 20;  // 4 MiB
 static __device__ __align__(256) unsigned char qsa_decode_scratch[kScratchBytes];
 
-void* g_scratch_ptr[64] = {nullptr};
+std::atomic<void*> g_scratch_ptr[64];  // zero-initialised (static storage)
 
 // Device address of the scratch array on the current device (looked up once per device).
 cudaError_t scratch_address(void** out) {
@@ -30,13 +34,13 @@ cudaError_t scratch_address(void** out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
+  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
     e = cudaGetSymbolAddress(&p, qsa_decode_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+    g_scratch_ptr[dev].store(p, std::memory_order_release);
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return cudaSuccess;
 }
 

@@ -705,21 +705,46 @@ size_t mat_bytes(const Geometry& g) {
 
 }  // namespace
 
+// Path resolution is pure geometry, so workspace sizes are computable on a host with no driver.
 int resolve_score_path(const Geometry& g, int requested) {
-  if (requested == 3 && !score_dec_supported(g)) return 2;
-  if (requested >= 1 && requested <= 3) return requested;
-  if (g.num_q <= 128 && score_dec_supported(g)) return 3;
+  switch (requested) {
+    case 1: case 2: case 4: return requested;
+    case 3: return score_dec_plan_ok(g) ? 3 : 2;
+    default: break;
+  }
+  if (g.num_q <= 128 && score_dec_plan_ok(g)) return 3;
   return g.num_q <= 256 ? 2 : 1;
 }
 
+// The fast Di = 128 kernels (tcgen05 prefill, split-list decode) load operands through tensor
+// maps.  Without the driver's encoder they cannot run, and a silent switch to the mma.sync
+// streaming kernel would be a large, invisible slowdown: the call reports it instead (path 4
+// asks for the streaming kernel explicitly).
+bool score_path_runnable(const Geometry& g, int path) {
+  const bool needs_tma = (path == 1 && g.Di == 128) || path == 3;
+  return !needs_tma || tmap_encode_fn() != nullptr;
+}
+
 size_t score_workspace_bytes(const Geometry& g, int path) {
-  if (path == 1) {
+  if (path == 1 || path == 4) {
     size_t n = (size_t)g.num_q * stream_cap(g.topk) * 8;
-    if (score_tc_supported(g)) n = std::max(n, score_tc_workspace_bytes(g));
+    if (path == 1 && g.Di == 128) n = std::max(n, score_tc_workspace_bytes(g));
     return n;
   }
   if (path == 3) return score_dec_workspace_bytes(g);
   return mat_bytes(g);
+}
+
+bool score_redo_offset(const Geometry& g, int path, size_t* off) {
+  if (path == 1 && g.Di == 128) {
+    *off = score_tc_redo_offset(g);
+    return true;
+  }
+  if (path == 3) {
+    *off = score_dec_redo_offset(g);
+    return true;
+  }
+  return false;
 }
 
 cudaError_t launch_score_topk(const Geometry& g, int path, const void* idx_q, const void* idx_w,
@@ -728,14 +753,14 @@ cudaError_t launch_score_topk(const Geometry& g, int path, const void* idx_q, co
   (void)ws_bytes;
   if (g.num_q == 0) return cudaSuccess;
   const ScoreArgs a = make_args(g, idx_q, idx_w, kcomp, sel, n_sel, sel_scores);
-  if (path == 1) {
-    if (score_tc_supported(g)) {
-      // tensor-core kernel first; the rows it flags are recomputed by the exact streaming kernel
-      int32_t* redo = nullptr;
-      cudaError_t e = launch_score_tc(a, g, ws, &redo, s);
-      if (e != cudaSuccess) return e;
-      return run_stream<128>(a, g, ws, s, redo);
-    }
+  if (path == 1 && g.Di == 128) {
+    // tensor-core kernel first; the rows it flags are recomputed by the exact streaming kernel
+    int32_t* redo = nullptr;
+    cudaError_t e = launch_score_tc(a, g, ws, &redo, s);
+    if (e != cudaSuccess) return e;
+    return run_stream<128>(a, g, ws, s, redo);
+  }
+  if (path == 1 || path == 4) {
     switch (g.Di) {
       case 32: return run_stream<32>(a, g, ws, s);
       case 64: return run_stream<64>(a, g, ws, s);

@@ -134,14 +134,15 @@ __device__ __forceinline__ void tma3d(uint32_t dst, const CUtensorMap* m, int x,
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn();
 
 // score_tc.cu: the tcgen05 kernel (Di = 128) used by the streaming path.
-bool score_tc_supported(const Geometry& g);
 size_t score_tc_workspace_bytes(const Geometry& g);
+size_t score_tc_redo_offset(const Geometry& g);  // byte offset of the redo flags [num_q]
 cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int32_t** redo_out,
                             cudaStream_t s);
 
 // score_dec.cu: decode-sized batches (split warp lists + exact merge; Di = 128).
-bool score_dec_supported(const Geometry& g);
+bool score_dec_plan_ok(const Geometry& g);        // the split-list plan fits (any driver)
 size_t score_dec_workspace_bytes(const Geometry& g);
+size_t score_dec_redo_offset(const Geometry& g);  // byte offset of the redo flags [num_q]
 cudaError_t launch_score_dec(const ScoreArgs& a, const Geometry& g, void* ws, int32_t** redo_out,
                              cudaStream_t s);
 

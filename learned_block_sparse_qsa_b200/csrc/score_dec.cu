@@ -791,9 +791,15 @@ __global__ void __launch_bounds__(DM_THREADS)
 
 }  // namespace
 
-bool score_dec_supported(const Geometry& g) {
+bool score_dec_plan_ok(const Geometry& g) {
   DecPlan p;
-  return g.Di == 128 && g.topk <= 512 && tmap_encode_fn() != nullptr && dec_plan(g, &p);
+  return g.Di == 128 && g.topk <= 512 && dec_plan(g, &p);
+}
+
+size_t score_dec_redo_offset(const Geometry& g) {
+  DecPlan p;
+  if (!dec_plan(g, &p)) return 0;
+  return stream_region(g) + r256((size_t)p.T * 4 * p.nl * p.lk * 8) + r256((size_t)p.T * 4 * pad2(p.nl) * 8);
 }
 
 size_t score_dec_workspace_bytes(const Geometry& g) {

@@ -505,10 +505,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
   return fn;
 }
 
-bool score_tc_supported(const Geometry& g) { return g.Di == 128 && tmap_encode_fn() != nullptr; }
+size_t score_tc_redo_offset(const Geometry& g) { return (size_t)g.num_q * 2 * TC_CAP * 8; }
 
 size_t score_tc_workspace_bytes(const Geometry& g) {
-  return (size_t)g.num_q * 2 * TC_CAP * 8 + ((size_t)g.num_q * 4 + 255) / 256 * 256;
+  return score_tc_redo_offset(g) + ((size_t)g.num_q * 4 + 255) / 256 * 256;
 }
 
 // Launch the tensor-core kernel; rows it could not settle are flagged in `redo` (a workspace
@@ -518,7 +518,7 @@ cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int
   auto enc = tmap_encode_fn();
   if (!enc) return cudaErrorNotSupported;
   u64* cand = static_cast<u64*>(ws);
-  int32_t* redo = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + (size_t)g.num_q * 2 * TC_CAP * 8);
+  int32_t* redo = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + score_tc_redo_offset(g));
   *redo_out = redo;
   CUtensorMap tmA, tmB;
   {

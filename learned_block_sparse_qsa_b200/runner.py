@@ -16,7 +16,8 @@ import torch
 
 from . import (QSA_OP_DENSE_ATTN_DECODE, QSA_OP_INDEX_SCORE_TOPK, QSA_OP_SPARSE_ATTN_DECODE,
                QsaBatch, QsaConfig, qsa_dense_attn_decode, qsa_dense_attn_prefill,
-               qsa_index_compress, qsa_index_score_topk, qsa_sparse_attn_decode,
+               qsa_index_compress, qsa_index_score_redo_flags, qsa_index_score_topk,
+               qsa_sparse_attn_decode,
                qsa_sparse_attn_prefill, qsa_workspace_size)
 
 
@@ -128,6 +129,19 @@ class QsaRunner:
         else:
             qsa_dense_attn_prefill(self.cfg, b, q, k_pool, v_pool, out, lse, stream)
         return out
+
+    def redo_flags(self, b: QsaBatch):
+        """Host copy (numpy int32 [num_q]) of the last selection's redo flags -- 1 where the exact
+        streaming kernel recomputed a row the fast kernel could not settle -- or None when the
+        resolved score path keeps none.  Synchronises the device."""
+        ws, n = self.workspace(b, QSA_OP_INDEX_SCORE_TOPK)
+        if ws is None:
+            return None
+        p = qsa_index_score_redo_flags(self.cfg, b, ws, n)
+        if p is None:
+            return None
+        off = p - ws.data_ptr()
+        return ws[off: off + 4 * b.num_q].view(torch.int32).cpu().numpy()
 
     def error_bits(self) -> int:
         return int(self.err.item())

@@ -77,6 +77,11 @@ class Run:
         self.torch.cuda.synchronize()
         return self
 
+    def redo_flags(self):
+        """The score call's redo flags (int32 [num_q], 1 = recomputed by the exact streaming
+        kernel) read from the runner's workspace, or None when the path keeps none."""
+        return self.runner.redo_flags(self.b)
+
     def numpy(self):
         t = self.torch
         return dict(sel=self.sel.cpu().numpy(), n_sel=self.n_sel.cpu().numpy(),
@@ -137,6 +142,41 @@ def oracle_dense_row(c: Config, integer: bool, r: int):
     return orc.dense_causal(h.q([r])[0], k, v, t)
 
 
+def positive_int_weights(w_bits: np.ndarray) -> np.ndarray:
+    """Head weights in {1, 2, 3}, from the generator's integer weights in [-3, 3] (|w| mod 3 + 1),
+    as bf16 bits.  Positive weights are what the pages' workloads use; with weights <= 0 a row's
+    scores collapse onto a few values and the fast kernel hands the row to the exact one."""
+    w = orc.bf16_to_f64(w_bits)
+    return orc.f64_to_bf16_bits(np.abs(w) % 3 + 1)
+
+
+def tc_redo_model(scores: np.ndarray, topk: int, nsamp: int, cap: int = 2048, tile: int = 128,
+                  sample_every: int = 32) -> bool:
+    """Whether the tensor-core indexer kernel hands a row to the exact streaming kernel, for a row
+    whose fp32 candidate scores are known exactly (integer inputs).  A model of the kernel's
+    branch, not of the method: each row is split into two column halves of every 128-block tile;
+    rows of more than 2 * cap candidates (and more than topk) take as threshold the smaller of the
+    two halves' 32nd-best score over the sampled tiles (tiles 0, 32, ..., 32 * (nsamp - 1));
+    every key at or above it is kept; the row is redone when a half keeps more than cap keys or
+    the row keeps fewer than min(topk, candidates)."""
+    lim = scores.shape[0]
+    if lim == 0:
+        return False
+    b = np.arange(lim)
+    half = (b % tile) // (tile // 2)
+    tau = -np.inf
+    if lim > topk and lim > 2 * cap:
+        sampled = ((b // tile) % sample_every == 0) & ((b // tile) // sample_every < nsamp)
+        thr = []
+        for hf in (0, 1):
+            v = np.sort(scores[sampled & (half == hf)])[::-1]
+            thr.append(v[31] if v.size >= 32 else -np.inf)
+        tau = min(thr)
+    keep = scores >= tau
+    n0, n1 = int(np.sum(keep & (half == 0))), int(np.sum(keep & (half == 1)))
+    return n0 > cap or n1 > cap or n0 + n1 < min(topk, lim)
+
+
 def kth_score(scores: np.ndarray, k: int) -> float:
     if scores.size == 0:
         return 0.0
@@ -189,5 +229,5 @@ def sample_rows(c: Config, n: int) -> list[int]:
     return sorted(set(np.linspace(0, c.num_q - 1, n).round().astype(int).tolist()))
 
 
-__all__ = ["CONFIGS", "Run", "host_kcomp", "score_bound", "oracle_select_row", "oracle_attend_row",
+__all__ = ["CONFIGS", "Run", "positive_int_weights", "tc_redo_model", "host_kcomp", "score_bound", "oracle_select_row", "oracle_attend_row",
            "oracle_dense_row", "check_selection", "check_attention", "sample_rows", "math"]

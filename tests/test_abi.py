@@ -64,7 +64,7 @@ def test_workspace_sizes_are_host_computable():
     ("block_tokens", 8, q.QSA_ERR_UNSUPPORTED), ("idx_heads", 2, q.QSA_ERR_UNSUPPORTED),
     ("head_dim", 96, q.QSA_ERR_UNSUPPORTED), ("topk_blocks", 0, q.QSA_ERR_UNSUPPORTED),
     ("topk_blocks", 513, q.QSA_ERR_UNSUPPORTED), ("num_q_heads", 6, q.QSA_ERR_INVALID_ARG),
-    ("page_tokens", 32, q.QSA_ERR_UNSUPPORTED), ("score_path", 4, q.QSA_ERR_INVALID_ARG)])
+    ("page_tokens", 32, q.QSA_ERR_UNSUPPORTED), ("score_path", 5, q.QSA_ERR_INVALID_ARG)])
 def test_invalid_config_rejected_before_launch(field, value, status):
     cfg = q.QsaConfig.make(32, 4, 128, 128)
     setattr(cfg, field, value)
@@ -94,6 +94,30 @@ def test_invalid_arguments_rejected_before_launch():
         q.qsa_sparse_attn_decode(cfg, b, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, 12,
                                  None, 0, stream=0)
     assert e.value.status == q.QSA_ERR_WORKSPACE
+
+
+def test_redo_flags_live_in_the_score_workspace():
+    """The redo-flag query is host arithmetic on the workspace address: flags for the tensor-core
+    and split-list paths, none for the materialised and plain streaming paths."""
+    b = mk_batch(num_q=16384, max_pages=16384, num_pages=16384, max_pos=1048575)
+    ws = 1 << 40
+    for path, has in [(1, True), (2, False), (4, False)]:
+        cfg = q.QsaConfig.make(32, 4, 128, 128, score_path=path)
+        n = q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK)
+        p = q.qsa_index_score_redo_flags(cfg, b, ws, n)
+        assert (p is not None) == has
+        if has:
+            assert ws <= p and p + 16384 * 4 <= ws + n
+    dec = mk_batch(num_q=16, batch=4, max_pages=16384, num_pages=65536, max_pos=1048575)
+    cfg = q.QsaConfig.make(32, 4, 128, 128)
+    n = q.qsa_workspace_size(cfg, dec, q.QSA_OP_INDEX_SCORE_TOPK)
+    p = q.qsa_index_score_redo_flags(cfg, dec, ws, n)
+    assert p is not None and ws <= p and p + 16 * 4 <= ws + n
+    with pytest.raises(q.QsaError) as e:
+        q.qsa_index_score_redo_flags(cfg, dec, ws, n - 256)
+    assert e.value.status == q.QSA_ERR_WORKSPACE
+    c32 = q.QsaConfig.make(4, 1, 64, 32, score_path=1)
+    assert q.qsa_index_score_redo_flags(c32, b, ws, 1 << 40) is None
 
 
 def test_selftest_rejects_limits_outside_range_before_launch():

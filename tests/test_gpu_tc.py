@@ -1,11 +1,15 @@
-"""GPU parity of the tensor-core (tcgen05) indexer path: exact on integer inputs, ragged multi-
-sequence row tiles, and the exact fallback for rows whose sampled threshold keeps too few keys."""
+"""GPU parity of the tensor-core (tcgen05) indexer path: exact on integer inputs on both of its
+branches (rows of at most 4,096 candidates keep every key; longer rows -- every row of a long-
+context chunk -- keep the keys at or above a threshold taken from a sample of tiles), ragged
+multi-sequence row tiles, and the exact fallback for rows the fast kernel cannot settle.  The
+redo flags the score call leaves in its workspace show which kernel produced each checked row."""
 import numpy as np
 import pytest
 
 from oracle import qsa_oracle as orc
-from qsa_synth import Config
-from tests.qsa_testlib import Run, check_attention, check_selection, host, host_kcomp, score_bound
+from qsa_synth import CONFIGS, Config
+from tests.qsa_testlib import (Run, check_attention, check_selection, host, host_kcomp,
+                               positive_int_weights, sample_rows, score_bound, tc_redo_model)
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -15,25 +19,86 @@ if not torch.cuda.is_available():
 TC_PREFILL = Config("tc_prefill_T8192_di128", "prefill", 1, 8192, 8192, 8, 2, 64, 4, 128, seed=0x7C01)
 
 
-def check_rows(run, rows, integer, topk=None):
+def check_rows(run, rows, integer, topk=None, w_bits=None, model=False):
+    """Selections of the given rows against the oracle.  w_bits: head weights [num_q, 4] that
+    replaced the generator's.  model=True (integer inputs only): also compare the row's redo flag
+    with tc_redo_model; returns the number of checked rows the fast kernel settled itself."""
     o = run.numpy()
     c = run.c
     topk = c.topk if topk is None else topk
     h = host(c, integer)
     q_seq, q_pos = h.rows()
+    redo = run.redo_flags() if model else None
+    settled = 0
     for r in rows:
         s, t = int(q_seq[r]), int(q_pos[r])
         kc = host_kcomp(c, integer, s)
-        iq, iw = h.idx_q([r])[0], h.idx_w([r])[0]
+        iq = h.idx_q([r])[0]
+        iw = h.idx_w([r])[0] if w_bits is None else w_bits[r]
         ref_sel, ref_s = orc.qsa_select(kc, iq, iw, t, topk)
         check_selection(o["sel"][r], o["n_sel"][r], o["sel_scores"][r], ref_sel, ref_s, t, topk,
                         integer, score_bound(kc, iq, iw, t // 4))
-    return o
+        if model:
+            tile = r // 128
+            last = min(c.num_q, tile * 128 + 128) - 1  # rows of one sequence, positions ascending
+            ntile = (int(q_pos[last]) // 4 + 127) // 128  # the CTA's tiles: its longest row
+            nsamp = (ntile + 31) // 32
+            want = tc_redo_model(ref_s, topk, nsamp)
+            assert bool(redo[r]) == want, (r, t, int(redo[r]), want)
+            settled += not want
+    return settled if model else o
+
+
+def run_positive_weights(c, **kw):
+    """Integer inputs with head weights in {1, 2, 3} (positive, as in the pages' workloads)."""
+    run = Run(c, integer=True, score_path=1, **kw)
+    w = positive_int_weights(host(c, True).idx_w(np.arange(c.num_q)))
+    run.di.idx_w.copy_(torch.from_numpy(w.view(np.int16)).view(torch.bfloat16))
+    return run.step(), w
 
 
 def test_tc_prefill_integer_exact_all_rows():
+    """Rows of at most 2,048 candidates: the keep-every-key branch, no row handed over."""
     run = Run(TC_PREFILL, integer=True, score_path=1).step()
     check_rows(run, range(TC_PREFILL.num_q), True)
+    assert run.runner.error_bits() == 0
+    assert not run.redo_flags().any()
+
+
+SAMPLED = Config("tc_sampled_chunk4096_ctx65536", "prefill", 1, 65536, 4096, 8, 2, 64, 4, 128,
+                 shuffle_pages=True, seed=0x7C04)
+
+
+def test_tc_sampled_threshold_integer_exact_all_rows():
+    """A 4,096-token chunk at 65,536 tokens of context: every row has 15,360-16,383 candidates,
+    so every row takes the sampled-threshold branch.  All rows bit-exact against the oracle, and
+    each row's redo flag equals the model of the branch, which settles every row here: the
+    checked selections are the tensor-core kernel's own."""
+    run, w = run_positive_weights(SAMPLED)
+    settled = check_rows(run, range(SAMPLED.num_q), True, w_bits=w, model=True)
+    assert settled == SAMPLED.num_q
+    assert run.runner.error_bits() == 0
+
+
+def test_tc_sampled_threshold_generator_weights_exact():
+    """The same chunk with the generator's weights in [-3, 3]: rows whose weights are all <= 0
+    have mostly tied scores and are handed to the exact kernel; every row is still exact and
+    every redo flag matches the model."""
+    run = Run(SAMPLED, integer=True, score_path=1).step()
+    rows = list(range(0, SAMPLED.num_q, 3)) + [SAMPLED.num_q - 1]
+    settled = check_rows(run, rows, True, model=True)
+    assert 0 < settled < len(rows)
+
+
+def test_tc_c2_integer_sampled_rows():
+    """The C2 chunk (16,384 tokens at 131,072) on integer inputs with positive weights: 256 rows
+    across the chunk bit-exact, each settled by the tensor-core kernel, and no row of the chunk
+    handed over."""
+    c = CONFIGS["C2"]
+    run, w = run_positive_weights(c)
+    rows = sample_rows(c, 256)
+    assert check_rows(run, rows, True, w_bits=w, model=True) == len(rows)
+    assert not run.redo_flags().any()
     assert run.runner.error_bits() == 0
 
 
@@ -90,12 +155,14 @@ def test_tc_fallback_on_decreasing_scores(ctx, n_new):
     qb = torch.tensor(q[0]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     wb = torch.ones(4).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     _, q_pos = host(c, True).rows()
+    redo = run.redo_flags()
     for r in list(range(0, c.num_q, 11)) + [c.num_q - 1]:
         t = int(q_pos[r])
         ref_sel, ref_s = orc.qsa_select(kc, qb, wb, t, c.topk)
         check_selection(o["sel"][r], o["n_sel"][r], o["sel_scores"][r], ref_sel, ref_s, t, c.topk, True)
         if t // 4 > 512:
             assert list(ref_sel[:-1]) == list(range(512))  # the earliest blocks win
+        assert bool(redo[r]) == (t // 4 > 4096)  # only the sampled branch is defeated
 
 
 def test_tc_decode_shaped_tile_with_four_sequences():

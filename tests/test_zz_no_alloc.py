@@ -48,3 +48,36 @@ def test_noalloc_rejects_split_count_beyond_scratch():
         q.qsa_sparse_attn_decode_noalloc(run.cfg, run.b, d.q, d.k_pool, d.v_pool, run.sel, run.n_sel,
                                          run.out, None, 64)
     assert e.value.status == q.QSA_ERR_WORKSPACE
+
+
+def test_noalloc_auto_split_count_lowered_to_fit():
+    """128 query heads of dim 128 (16 per KV head): the automatic split count of the workspace
+    form would need more than the 4 MiB of library scratch, so the allocation-free form lowers it
+    to the largest count that fits.  Its output must equal the workspace form run at that count
+    (same kernels, same split: bit for bit), twice in a row."""
+    import learned_block_sparse_qsa_b200 as q
+
+    c = Config("noalloc_g16", "decode", 1, 8192, 4, 128, 8, 128, 4, 128, shuffle_pages=True,
+               seed=0x0A13)
+    run = Run(c, integer=False).step(splits=1)
+    auto = q.qsa_workspace_size(run.cfg, run.b, q.QSA_OP_SPARSE_ATTN_DECODE, 0)
+    assert auto > 4 << 20  # the automatic count does not fit: the lowering loop runs
+    fit = max(s for s in range(1, 65)
+              if q.qsa_workspace_size(run.cfg, run.b, q.QSA_OP_SPARSE_ATTN_DECODE, s) <= 4 << 20)
+    assert fit > 1
+    d = run.di
+    ref = torch.empty_like(run.out)
+    ref_lse = torch.empty_like(run.lse)
+    ws, n = run.runner.workspace(run.b, q.QSA_OP_SPARSE_ATTN_DECODE, fit)
+    q.qsa_sparse_attn_decode(run.cfg, run.b, d.q, d.k_pool, d.v_pool, run.sel, run.n_sel, ref,
+                             ref_lse, fit, ws, n)
+    for _ in range(2):
+        out = torch.full_like(run.out, float("nan"))
+        lse = torch.full_like(run.lse, float("nan"))
+        q.qsa_sparse_attn_decode_noalloc(run.cfg, run.b, d.q, d.k_pool, d.v_pool, run.sel,
+                                         run.n_sel, out, lse, 0)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+        assert torch.equal(lse, ref_lse)
+    assert torch.allclose(run.out.float(), ref.float(), atol=ATTN_ATOL, rtol=ATTN_RTOL)
+    assert run.runner.error_bits() == 0
