@@ -209,6 +209,23 @@ qsa_status_t qsa_dense_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* b
                                    void* out, float* lse, int32_t num_splits, void* workspace,
                                    size_t ws_bytes, qsa_stream_t stream);
 
+/* The indexer's dense-distillation signal (section "The indexer is trained, not bolted on": the
+ * indexer first learned from the full-attention distribution, token-level attention pooled into
+ * blocks being the teacher).  For every query row at position t: the teacher is the dense causal
+ * softmax attention of all Hq core heads over positions 0..t (softmax scale and head mapping as in
+ * the core attention), summed over the 4 tokens of each candidate block b < t/4 and over the
+ * heads, renormalised over the candidates; the student is the softmax over the same blocks of the
+ * indexer scores s_b(t) (the selection scores); kl[i] (float [num_q]) = KL(teacher || student) in
+ * nats, 0 when t < 4 and NaN for a row whose sequence or position is invalid (flagged).
+ * Optional outputs: lse (float [num_q, Hq], natural-log normaliser of each head's dense softmax)
+ * and teacher (float [num_q, ld], ld >= max_pos/4: the teacher distribution, entries b >= t/4
+ * untouched).  Needs keys of positions 0..t in k_pool and the compressed keys of blocks < t/4;
+ * reads no values.  No workspace.  A dense computation (two passes of q.k over the context). */
+qsa_status_t qsa_index_distill_kl(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                  const void* q, const void* k_pool, const void* idx_q,
+                                  const void* idx_w, const void* kcomp_pool, float* kl, float* lse,
+                                  float* teacher, int64_t ld, qsa_stream_t stream);
+
 /* No counterpart in the article: a self-test of failure detection.  Every pipelined kernel waits
  * on mbarriers with a bounded wait that, when it runs out, sets QSA_DEVERR_TIMEOUT in *err_flag
  * and lets the kernel return instead of hanging.  This call launches one CTA that waits, with that

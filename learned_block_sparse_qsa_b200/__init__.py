@@ -87,6 +87,8 @@ _SIGS = {
                                          c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
     "qsa_sparse_attn_decode_noalloc": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p,
                                                   c_void_p, c_void_p, c_void_p, c_int32, c_void_p]),
+    "qsa_index_distill_kl": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
     "qsa_dense_attn_prefill": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_void_p]),
     "qsa_dense_attn_decode": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -170,6 +172,15 @@ def qsa_sparse_attn_decode_noalloc(cfg, batch, q, k_pool, v_pool, sel, n_sel, ou
                                                _p(k_pool), _p(v_pool), _p(sel), _p(n_sel), _p(out),
                                                _p(lse), int(num_splits), _stream(stream)),
            "qsa_sparse_attn_decode_noalloc")
+
+
+def qsa_index_distill_kl(cfg, batch, q, k_pool, idx_q, idx_w, kcomp_pool, kl, lse=None,
+                         teacher=None, ld=0, stream=None):
+    """Per-row KL(block-pooled dense attention || indexer softmax); see include/qsa.h."""
+    _check(_lib.qsa_index_distill_kl(ctypes.byref(cfg), ctypes.byref(batch), _p(q), _p(k_pool),
+                                     _p(idx_q), _p(idx_w), _p(kcomp_pool), _p(kl), _p(lse),
+                                     _p(teacher), int(ld), _stream(stream)),
+           "qsa_index_distill_kl")
 
 
 def qsa_dense_attn_prefill(cfg, batch, q, k_pool, v_pool, out, lse=None, stream=None):

@@ -220,6 +220,22 @@ qsa_status_t qsa_sparse_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* 
                                            lse, s, workspace, (cudaStream_t)stream));
 }
 
+qsa_status_t qsa_index_distill_kl(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                  const void* q, const void* k_pool, const void* idx_q,
+                                  const void* idx_w, const void* kcomp_pool, float* kl, float* lse,
+                                  float* teacher, int64_t ld, qsa_stream_t stream) {
+  Geometry g;
+  qsa_status_t st = make_geometry(cfg, batch, &g, true);
+  if (st != QSA_OK || g.num_q == 0) return st;
+  if (!q || !k_pool || !idx_q || !idx_w || !kcomp_pool || !kl) return QSA_ERR_INVALID_ARG;
+  if (teacher && ld < g.max_pos / 4) return QSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k_pool) |
+       reinterpret_cast<uintptr_t>(idx_q) | reinterpret_cast<uintptr_t>(kcomp_pool)) & 15)
+    return QSA_ERR_INVALID_ARG;
+  return from_cuda(qsa::launch_distill(g, q, k_pool, idx_q, idx_w, kcomp_pool, kl, lse, teacher,
+                                       ld, (cudaStream_t)stream));
+}
+
 qsa_status_t qsa_dense_attn_prefill(const qsa_config_t* cfg, const qsa_batch_t* batch,
                                     const void* q, const void* k_pool, const void* v_pool,
                                     void* out, float* lse, qsa_stream_t stream) {

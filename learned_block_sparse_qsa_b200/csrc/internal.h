@@ -48,6 +48,11 @@ cudaError_t launch_dense_attn(const Geometry& g, const void* q, const void* k_po
                               const void* v_pool, void* out, float* lse, int splits, void* ws,
                               cudaStream_t s);
 
+// distill.cu
+cudaError_t launch_distill(const Geometry& g, const void* q, const void* k_pool, const void* idx_q,
+                           const void* idx_w, const void* kcomp, float* kl, float* lse,
+                           float* teacher, int64_t ld, cudaStream_t s);
+
 // combine (attn.cu): merge split partials [num_q, splits, Hq] of (o fp32 [D], lse2) -> bf16
 cudaError_t launch_combine(const Geometry& g, const float* part_o, const float* part_lse,
                            int splits, void* out, float* lse, cudaStream_t s);
