@@ -473,9 +473,45 @@ def dense_time_ms(w: Workload, decode: bool, reps: int, flush=None):
 
 # ------------------------------------------------------------------------------------ oracle
 
+def _oracle_rows(h, kc, rows, workers: int):
+    """Wall seconds of the oracle's selection and attention for the given query rows, run on
+    `workers` host threads (BLAS limited to one thread each).  Inputs are generated outside the
+    timed parts: the rows' queries first, then the K/V rows the selections name."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from oracle import qsa_oracle as orc
+
+    _, q_pos = h.rows()
+    rows = list(rows)
+    iq, iw, qq = h.idx_q(rows), h.idx_w(rows), h.q(rows)
+    q_seq = h.rows()[0]
+    with threadpool_limits(limits=1), ThreadPoolExecutor(max_workers=workers) as ex:
+        def sel(i):
+            t = int(q_pos[rows[i]])
+            s, _ = orc.qsa_select(kc[int(q_seq[rows[i]])], iq[i], iw[i], t)
+            return orc.expand(s, t)
+
+        t0 = time.perf_counter()
+        pos = list(ex.map(sel, range(len(rows))))
+        t_sel = time.perf_counter() - t0
+        kv = [h.kv(int(q_seq[r]), p) for r, p in zip(rows, pos)]   # input regeneration, untimed
+        t0 = time.perf_counter()
+        list(ex.map(lambda i: orc.attend(qq[i], *kv[i]), range(len(rows))))
+        t_att = time.perf_counter() - t0
+    return t_sel + t_att
+
+
+def oracle_workers() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
 def oracle_prefill_baseline(rows_per_step: int, steps: int):
     """The fp64 oracle on the host cores, on a bounded sample of the prefill workload: the
-    chunk's compression once, then selection + attention for evenly spaced query rows."""
+    chunk's compression, then selection + attention of evenly spaced query rows on one host
+    thread per core."""
     import numpy as np
 
     from oracle import qsa_oracle as orc
@@ -488,37 +524,43 @@ def oracle_prefill_baseline(rows_per_step: int, steps: int):
     t0 = time.perf_counter()
     kc_chunk = orc.compress(chunk_keys)
     t_compress = time.perf_counter() - t0
-    kc = np.concatenate([kc_prefix, kc_chunk])
+    kc = {0: np.concatenate([kc_prefix, kc_chunk])}
     n = rows_per_step * steps
     rows = np.linspace(0, c.num_q - 1, n).round().astype(int)
-    _, q_pos = h.rows()
-    iq, iw, qq = h.idx_q(rows), h.idx_w(rows), h.q(rows)
-    t_rows = 0.0
-    per_step = []
-    for i, r in enumerate(rows):
-        t = int(q_pos[r])
-        a = time.perf_counter()
-        sel, _ = orc.qsa_select(kc, iq[i], iw[i], t)
-        pos = orc.expand(sel, t)
-        b = time.perf_counter()
-        k, v = h.kv(0, pos)                                      # input regeneration, not timed
-        c0 = time.perf_counter()
-        orc.attend(qq[i], k, v)
-        e = time.perf_counter()
-        t_rows += (b - a) + (e - c0)
-        per_step.append((b - a) + (e - c0))
+    workers = oracle_workers()
+    t_rows = _oracle_rows(h, kc, rows, workers)
     per_token = t_compress / c.num_q + t_rows / n
-    try:
-        from threadpoolctl import threadpool_info
-
-        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:  # pragma: no cover
-        cores = os.cpu_count() or 1
-    return dict(value=1.0 / per_token, unit="tok/s", cores=int(cores), kind="oracle",
+    return dict(value=1.0 / per_token, unit="tok/s", cores=workers, kind="oracle",
                 sample=f"{n} evenly spaced query rows of the {c.num_q}-token chunk at "
-                       f"{c.ctx}-token context (selection + attention each) plus the chunk's "
-                       f"compression; tok/s extrapolated from seconds per token",
+                       f"{c.ctx}-token context (selection + attention each, {workers} threads, "
+                       f"BLAS one thread each) plus the chunk's compression; tok/s extrapolated "
+                       f"from seconds per token",
                 seconds=t_compress + t_rows)
+
+
+def oracle_decode_baseline():
+    """The fp64 oracle on one sequence of the decode step: its new block's compression and the
+    selection + attention of its 4 query positions on 4 host threads; the step (4 sequences, one
+    after the other) is extrapolated as 4 times that."""
+    import numpy as np
+
+    from oracle import qsa_oracle as orc
+    from qsa_synth import CONFIGS, HostInputs
+
+    c = CONFIGS[DECODE]
+    h = HostInputs(c)
+    kc_prefix = orc.compress(h.idx_k(0, 0, c.ctx_start))       # setup, not timed
+    new_keys = h.idx_k(0, c.ctx_start, c.ctx)
+    t0 = time.perf_counter()
+    kc_new = orc.compress(new_keys)
+    t_compress = time.perf_counter() - t0
+    kc = {0: np.concatenate([kc_prefix, kc_new])}
+    t_rows = _oracle_rows(h, kc, range(c.n_new), c.n_new)
+    us = (t_compress + t_rows) * c.batch * 1e6
+    return dict(value=us, unit="us/step", cores=c.n_new, kind="oracle",
+                sample=f"sequence 0 of {c.batch}: its new block's compression and its {c.n_new} "
+                       f"query positions (selection + attention, {c.n_new} threads) at "
+                       f"{c.ctx}-token context; the step is extrapolated as {c.batch} x that")
 
 
 # ------------------------------------------------------------------------------------ main
@@ -605,7 +647,7 @@ def main():
                          peak=peaks["hbm"], kernel_file="compress.cu"),
         "score_topk": dict(ms=stage_ms["score_topk"], bound="tensor", unit="TFLOP/s",
                            achieved=work["score_flops"] / (stage_ms["score_topk"] * 1e-3) / 1e12,
-                           peak=peaks["tf_sus"], kernel_file="score.cu"),
+                           peak=peaks["tf"], kernel_file="score_tc.cu"),
         "sparse_attn": dict(ms=stage_ms["sparse_attn"], bound="hbm", unit="GB/s",
                             achieved=work["attn_bytes"] / (stage_ms["sparse_attn"] * 1e-3) / 1e9,
                             peak=peaks["hbm"], kernel_file="attn.cu"),
@@ -618,16 +660,16 @@ def main():
                   "sparse_attn": work["attn_bytes"]}[dom]
     roofline = {"bound": ds["bound"], "achieved": ds["achieved"], "peak": ds["peak"], "unit": ds["unit"],
                 "frac": ds["frac"], "kernel": dom, "work_per_launch": per_launch,
-                "peak_source": peaks["src"] + (" sustained" if ds["bound"] == "tensor" else ""),
+                "peak_source": peaks["src"] + (" burst" if ds["bound"] == "tensor" else ""),
                 "traffic": traffic_for(ds["kernel_file"], f"{dom}@{PREFILL}")}
-    path_roof_ms = (work["compress_bytes"] / (peaks["hbm"] * 1e9) + work["score_flops"] / (peaks["tf_sus"] * 1e12)
+    path_roof_ms = (work["compress_bytes"] / (peaks["hbm"] * 1e9) + work["score_flops"] / (peaks["tf"] * 1e12)
                     + work["attn_bytes"] / (peaks["hbm"] * 1e9)) * 1e3
     log(f"prefill {c.name}: {ms_step:.3f} ms/step, {value / 1e6:.3f} M tok/s, stages "
         + ", ".join(f"{k} {v['ms']:.3f} ms ({100 * v['frac']:.1f}% {v['bound']})" for k, v in stages.items()))
     e2e_ms, h2d, d2h = e2e_prefill(w, max(3, args.steps), 2)
     e2e_ms = max_over_ranks(e2e_ms, dist)
     log(f"prefill e2e {e2e_ms:.3f} ms/step")
-    dense_ms = dense_time_ms(w, False, 1)
+    dense_ms = dense_time_ms(w, False, 3)
     log(f"dense prefill {dense_ms:.1f} ms ({work['dense_flops'] / (dense_ms * 1e-3) / 1e12:.1f} TFLOP/s)")
     del w
     torch.cuda.empty_cache()
@@ -662,10 +704,13 @@ def main():
     del wd
     torch.cuda.empty_cache()
 
-    cpu = None
+    cpu = dcpu = None
     if rank == 0 and world == 1:
-        base = oracle_prefill_baseline(rows_per_step=8, steps=4)
+        base = oracle_prefill_baseline(rows_per_step=16, steps=4)
         cpu = {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        dcpu = oracle_decode_baseline()
+        log(f"oracle: prefill {cpu['value']:.2f} tok/s on {cpu['cores']} threads; decode "
+            f"{dcpu['value'] / 1e3:.1f} ms/step")
 
     if rank == 0:
         line = {
@@ -700,6 +745,7 @@ def main():
                        "stages_us": {k: v["ms"] * 1000 for k, v in dstages.items()},
                        "stages": dstages, "path_roofline_us": dpath_roof_us,
                        "path_roofline_frac": dpath_roof_us / graph_us,
+                       "cpu_baseline": dcpu,
                        "e2e": {"value": d_e2e_us, "unit": "us/step", "h2d_bytes_per_step": dh2d,
                                "d2h_bytes_per_step": dd2h},
                        "gpu_launches_per_step": 5},

@@ -7,9 +7,9 @@
  * inputs of many GiB are created where they are used.  The numpy twin in
  * qsa_synth/__init__.py reproduces any element bit for bit on the host.
  *
- * All pointers are device pointers owned by the caller; `stream` is a
- * cudaStream_t (NULL = legacy default stream).  Calls are asynchronous and
- * return a cudaError_t value (0 = success) from the launch.
+ * Pointers are device pointers owned by the caller, except in the host fill;
+ * `stream` is a cudaStream_t (NULL = legacy default stream).  Device calls are
+ * asynchronous and return a cudaError_t value (0 = success) from the launch.
  */
 #ifndef QSA_SYNTH_H
 #define QSA_SYNTH_H
@@ -34,6 +34,11 @@ int qsyn_fill_linear(void* out, int64_t n, int64_t offset, uint64_t seed, uint64
 int qsyn_fill_paged(void* pool, int64_t num_pages, int page_tokens, int row_elems,
                     const int32_t* page_owner, int max_pages, int64_t seq_stride, uint64_t seed,
                     uint64_t tid, int dist, void* stream);
+
+/* Host memory: out bf16 [nrows, width]; row r holds value(seed, tid, starts[r] + e), e < width.
+ * Runs on `threads` host threads (<= 0: all cores).  Returns 0, or 1 for a NULL pointer. */
+int qsyn_fill_rows_host(void* out, const int64_t* starts, int64_t nrows, int64_t width,
+                        uint64_t seed, uint64_t tid, int dist, int threads);
 
 #ifdef __cplusplus
 }

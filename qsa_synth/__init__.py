@@ -88,6 +88,48 @@ def values_bf16(seed: int, tid: int, idx, dist: int) -> np.ndarray:
     raise ValueError(dist)
 
 
+_HOST_LIB = None
+
+
+def _host_lib():
+    """libqsa_synth.so's host fill (the same values, computed by C++ threads), or None when the
+    library has not been built; the numpy path above is then used."""
+    global _HOST_LIB
+    if _HOST_LIB is None:
+        import ctypes
+        import os
+
+        path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqsa_synth.so")
+        lib = False
+        if os.path.exists(path):
+            try:
+                lib = ctypes.CDLL(path)
+                f = lib.qsyn_fill_rows_host
+                f.restype = ctypes.c_int
+                f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                              ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int, ctypes.c_int]
+            except (OSError, AttributeError):
+                lib = False
+        _HOST_LIB = lib
+    return _HOST_LIB or None
+
+
+def rows_bf16(seed: int, tid: int, starts, width: int, dist: int) -> np.ndarray:
+    """bf16 bits [len(starts), width]: row r holds elements starts[r] .. starts[r] + width - 1 of
+    stream (seed, tid).  Equal to values_bf16 of those indices (checked by tests/test_synth.py)."""
+    starts = np.ascontiguousarray(starts, dtype=np.int64).reshape(-1)
+    lib = _host_lib()
+    if lib is None or starts.size * width < 4096:
+        idx = starts[:, None] + np.arange(width, dtype=np.int64)[None, :]
+        return values_bf16(seed, tid, idx.reshape(-1), dist).reshape(starts.size, width)
+    out = np.empty((starts.size, width), dtype=np.uint16)
+    rc = lib.qsyn_fill_rows_host(out.ctypes.data, starts.ctypes.data, starts.size, width, seed, tid,
+                                 dist, 0)
+    if rc != 0:
+        raise RuntimeError("qsyn_fill_rows_host failed")
+    return out
+
+
 def values_f32(seed: int, tid: int, idx, dist: int) -> np.ndarray:
     return bf16_bits_to_f32(values_bf16(seed, tid, idx, dist))
 
@@ -262,8 +304,7 @@ class HostInputs:
 
     # ---- tensors (bf16 bit patterns, uint16)
     def _lin(self, tid, dist, starts, width):
-        idx = (np.asarray(starts, dtype=np.int64)[:, None] + np.arange(width, dtype=np.int64)[None, :])
-        return values_bf16(self.cfg.seed, tid, idx.reshape(-1), dist).reshape(len(starts), width)
+        return rows_bf16(self.cfg.seed, tid, starts, width, dist)
 
     def q(self, rows) -> np.ndarray:
         c = self.cfg
@@ -295,12 +336,8 @@ class HostInputs:
         """Raw indexer keys of positions [pos0, pos1) of sequence s: bf16 [n, Di]."""
         c = self.cfg
         n = pos1 - pos0
-        out = np.empty((n, c.Di), dtype=np.uint16)
-        step = max(1, (1 << 22) // c.Di)
-        for a in range(0, n, step):
-            b = min(n, a + step)
-            idx = (s * c.ctx + pos0 + a) * c.Di + np.arange((b - a) * c.Di, dtype=np.int64)
-            out[a:b] = values_bf16(c.seed, TID_IDXK, idx, self.dist["idx_k"]).reshape(b - a, c.Di)
+        starts = (s * c.ctx + pos0 + np.arange(n, dtype=np.int64)) * c.Di
+        out = rows_bf16(c.seed, TID_IDXK, starts, c.Di, self.dist["idx_k"])
         nd = self.needles()
         if nd["blocks"]:
             for j, blk in enumerate(nd["blocks"][s]):

@@ -29,7 +29,7 @@ CASES = {
                                    needles=8, shuffle_pages=True, seed=0xD151),
     "g16_32q2kv_d64_di64": Config("distill_g16", "prefill", 1, 3000, 200, 32, 2, 64, 4, 64,
                                   shuffle_pages=True, seed=0xD152),
-    "g1_8q8kv_d64_di128": Config("distill_g1", "prefill", 1, 2500, 150, 8, 8, 64, 4, 128,
+    "g1_8q8kv_d64_di128": Config("distill_g1", "prefill", 1, 2500, 152, 8, 8, 64, 4, 128,
                                  seed=0xD153),
 }
 

@@ -64,3 +64,18 @@ def test_needles_have_cosine_point_eight():
     blk = int(nd["blocks"][s][0])
     rows = h.idx_k(s, 4 * blk, 4 * blk + 4)
     assert np.all(rows == rows[0]) and np.array_equal(rows[0], nd["key_rows"][s][0])
+
+
+def test_host_fill_equals_numpy_generator():
+    """The C++ host fill of libqsa_synth.so returns the numpy generator's bits, for every
+    distribution and for rows starting at arbitrary indices."""
+    if qs._host_lib() is None:
+        import pytest
+
+        pytest.skip("libqsa_synth.so not built")
+    rng = np.random.default_rng(5)
+    starts = rng.integers(0, 1 << 40, 300)
+    for dist in (qs.NORMAL, qs.UNIFORM, qs.INT3):
+        got = qs.rows_bf16(11, 4, starts, 129, dist)
+        idx = starts[:, None] + np.arange(129)[None, :]
+        assert np.array_equal(got, qs.values_bf16(11, 4, idx.reshape(-1), dist).reshape(300, 129))
