@@ -209,6 +209,20 @@ qsa_status_t qsa_dense_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* b
                                    void* out, float* lse, int32_t num_splits, void* workspace,
                                    size_t ws_bytes, qsa_stream_t stream);
 
+/* Backward of steps (d)+(e) with the selection held fixed (section "The indexer is trained, not
+ * bolted on": after the dense warm-up the indexer and the backbone trained together through the
+ * sparse layer; a top-k choice has no gradient).  Inputs as for qsa_sparse_attn_prefill plus the
+ * forward's out (bf16 [num_q, Hq, D]) and lse (float [num_q, Hq], natural log) and the upstream
+ * gradient dout (bf16 [num_q, Hq, D]).  Outputs: dq (float [num_q, Hq, D], written) and the
+ * gradients of the key and value caches, dk_pool and dv_pool (float [num_pages, 64, Hkv, D], the
+ * caches' layout in fp32): ADDED to, since every row that selected a block contributes to its
+ * positions -- zero them first.  Hq/Hkv <= 8 (QSA_ERR_UNSUPPORTED otherwise).  No workspace. */
+qsa_status_t qsa_sparse_attn_backward(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                      const void* q, const void* k_pool, const void* v_pool,
+                                      const int32_t* sel, const int32_t* n_sel, const void* out,
+                                      const float* lse, const void* dout, float* dq,
+                                      float* dk_pool, float* dv_pool, qsa_stream_t stream);
+
 /* The indexer's dense-distillation signal (section "The indexer is trained, not bolted on": the
  * indexer first learned from the full-attention distribution, token-level attention pooled into
  * blocks being the teacher).  For every query row at position t: the teacher is the dense causal

@@ -87,6 +87,9 @@ _SIGS = {
                                          c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
     "qsa_sparse_attn_decode_noalloc": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p,
                                                   c_void_p, c_void_p, c_void_p, c_int32, c_void_p]),
+    "qsa_sparse_attn_backward": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_void_p, c_void_p]),
     "qsa_index_distill_kl": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
     "qsa_dense_attn_prefill": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -172,6 +175,16 @@ def qsa_sparse_attn_decode_noalloc(cfg, batch, q, k_pool, v_pool, sel, n_sel, ou
                                                _p(k_pool), _p(v_pool), _p(sel), _p(n_sel), _p(out),
                                                _p(lse), int(num_splits), _stream(stream)),
            "qsa_sparse_attn_decode_noalloc")
+
+
+def qsa_sparse_attn_backward(cfg, batch, q, k_pool, v_pool, sel, n_sel, out, lse, dout, dq,
+                             dk_pool, dv_pool, stream=None):
+    """Gradients of the sparse attention (dq written; dk_pool, dv_pool accumulated)."""
+    _check(_lib.qsa_sparse_attn_backward(ctypes.byref(cfg), ctypes.byref(batch), _p(q), _p(k_pool),
+                                         _p(v_pool), _p(sel), _p(n_sel), _p(out), _p(lse),
+                                         _p(dout), _p(dq), _p(dk_pool), _p(dv_pool),
+                                         _stream(stream)),
+           "qsa_sparse_attn_backward")
 
 
 def qsa_index_distill_kl(cfg, batch, q, k_pool, idx_q, idx_w, kcomp_pool, kl, lse=None,

@@ -220,6 +220,23 @@ qsa_status_t qsa_sparse_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* 
                                            lse, s, workspace, (cudaStream_t)stream));
 }
 
+qsa_status_t qsa_sparse_attn_backward(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                      const void* q, const void* k_pool, const void* v_pool,
+                                      const int32_t* sel, const int32_t* n_sel, const void* out,
+                                      const float* lse, const void* dout, float* dq,
+                                      float* dk_pool, float* dv_pool, qsa_stream_t stream) {
+  Geometry g;
+  qsa_status_t st = sparse_common(cfg, batch, q, k_pool, v_pool, sel, n_sel, const_cast<void*>(out), &g);
+  if (st != QSA_OK || g.num_q == 0) return st;
+  if (!lse || !dout || !dq || !dk_pool || !dv_pool) return QSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(dout) | reinterpret_cast<uintptr_t>(dk_pool) |
+       reinterpret_cast<uintptr_t>(dv_pool)) & 15)
+    return QSA_ERR_INVALID_ARG;
+  if (g.G > 8) return QSA_ERR_UNSUPPORTED;
+  return from_cuda(qsa::launch_sparse_attn_bwd(g, q, k_pool, v_pool, sel, n_sel, out, lse, dout, dq,
+                                               dk_pool, dv_pool, (cudaStream_t)stream));
+}
+
 qsa_status_t qsa_index_distill_kl(const qsa_config_t* cfg, const qsa_batch_t* batch,
                                   const void* q, const void* k_pool, const void* idx_q,
                                   const void* idx_w, const void* kcomp_pool, float* kl, float* lse,

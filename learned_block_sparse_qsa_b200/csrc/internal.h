@@ -48,6 +48,12 @@ cudaError_t launch_dense_attn(const Geometry& g, const void* q, const void* k_po
                               const void* v_pool, void* out, float* lse, int splits, void* ws,
                               cudaStream_t s);
 
+// attn_bwd.cu
+cudaError_t launch_sparse_attn_bwd(const Geometry& g, const void* q, const void* k_pool,
+                                   const void* v_pool, const int32_t* sel, const int32_t* n_sel,
+                                   const void* out, const float* lse, const void* dout, float* dq,
+                                   float* dk_pool, float* dv_pool, cudaStream_t s);
+
 // distill.cu
 cudaError_t launch_distill(const Geometry& g, const void* q, const void* k_pool, const void* idx_q,
                            const void* idx_w, const void* kcomp, float* kl, float* lse,
