@@ -71,7 +71,8 @@ typedef enum qsa_status {
 typedef enum qsa_op {
   QSA_OP_INDEX_SCORE_TOPK = 1,
   QSA_OP_SPARSE_ATTN_DECODE = 2,
-  QSA_OP_DENSE_ATTN_DECODE = 3
+  QSA_OP_DENSE_ATTN_DECODE = 3,
+  QSA_OP_MERGE_CANDIDATES = 4 /* num_splits = number of parts */
 } qsa_op_t;
 
 typedef struct qsa_config {
@@ -208,6 +209,52 @@ qsa_status_t qsa_dense_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* b
                                    const void* q, const void* k_pool, const void* v_pool,
                                    void* out, float* lse, int32_t num_splits, void* workspace,
                                    size_t ws_bytes, qsa_stream_t stream);
+
+/* ---- Context parallelism: one sequence's context split across ranks (not in the article, which
+ * measures one accelerator; built so that a million-token context can be shared by several).
+ * Rank r holds positions [start_r, start_r + len_r) of the sequence (multiples of 64: whole
+ * pages) with a local page table of len_r/64 + 1 columns (the last one may name any valid page).
+ * Per step: (1) qsa_cp_shard_positions gives each row's local positions; (2) the rank runs
+ * qsa_index_score_topk with q_pos = pos_sel and its local tables: the exact best candidates of its
+ * shard, in local block ids (its tail entry is ignored later); (3) the callers all-gather the ranks'
+ * sel and sel_scores; (4) qsa_index_merge_candidates gives the global selection -- equal to the
+ * single-accelerator one, because every global winner is a winner of its own shard -- and the
+ * winners inside this rank's shard in local ids; (5) the rank attends over those with
+ * q_pos = pos_attn (qsa_sparse_attn_prefill or _decode, lse requested); (6) the callers all-gather
+ * the partial outputs and log-sum-exps and qsa_attn_merge_partials combines them. */
+
+/* Local positions of the rows for the shard [shard_start, shard_start + shard_len) (device int32
+ * [num_q] each): pos_sel = t - start clamped to [0, len] (len: every block of a shard that ends
+ * before t is a candidate; 0: none of a shard that starts after t); pos_attn = t - start clamped
+ * to [0, len - 1].  start and len: multiples of 64. */
+qsa_status_t qsa_cp_shard_positions(const int32_t* q_pos, int32_t num_q, int32_t shard_start,
+                                    int32_t shard_len, int32_t* pos_sel, int32_t* pos_attn,
+                                    qsa_stream_t stream);
+
+/* Exact merge of nparts candidate lists (section "A million-token window with a selective view":
+ * the best 512 blocks of the whole context plus the tail).  part_sel / part_scores: device
+ * [nparts, num_q, topk+1] as qsa_index_score_topk wrote them on each part (local block ids; +inf
+ * scores mark tails and are skipped, -1 / NaN padding too); part_block_lo: HOST int32 [nparts], the
+ * first global block of each part.  batch carries the GLOBAL q_seq / q_pos.  Writes the global
+ * sel / n_sel / sel_scores (as qsa_index_score_topk would) and, for this rank's blocks
+ * [block_lo, block_hi), local_sel (int32 [num_q, topk+1], local ids ascending, the tail included
+ * when it lies there, -1 padded) and local_n (int32 [num_q]).  workspace:
+ * qsa_workspace_size(..., QSA_OP_MERGE_CANDIDATES, nparts, ...) bytes.  nparts <= 64. */
+qsa_status_t qsa_index_merge_candidates(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                        int32_t nparts, const int32_t* part_sel,
+                                        const float* part_scores, const int32_t* part_block_lo,
+                                        int32_t block_lo, int32_t block_hi, int32_t* sel,
+                                        int32_t* n_sel, float* sel_scores, int32_t* local_sel,
+                                        int32_t* local_n, void* workspace, size_t ws_bytes,
+                                        qsa_stream_t stream);
+
+/* out (bf16 [num_q, Hq, D]) and lse (float [num_q, Hq] or NULL) from nparts partial attentions
+ * over disjoint position sets: part_out bf16 [nparts, num_q, Hq, D], part_lse float
+ * [nparts, num_q, Hq] (natural log; -inf for an empty part): out = sum_p exp(lse_p - L) o_p with
+ * L = log sum_p exp(lse_p). */
+qsa_status_t qsa_attn_merge_partials(int32_t nparts, int32_t num_q, int32_t num_q_heads,
+                                     int32_t head_dim, const void* part_out, const float* part_lse,
+                                     void* out, float* lse, qsa_stream_t stream);
 
 /* Backward of steps (d)+(e) with the selection held fixed (section "The indexer is trained, not
  * bolted on": after the dense warm-up the indexer and the backbone trained together through the

@@ -24,6 +24,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA = 0, 1, 2, 3, 4
 QSA_OP_INDEX_SCORE_TOPK, QSA_OP_SPARSE_ATTN_DECODE, QSA_OP_DENSE_ATTN_DECODE = 1, 2, 3
+QSA_OP_MERGE_CANDIDATES = 4
 DEVERR = {"SEQ": 1, "POS": 2, "PAGE": 4, "GROUP": 8, "SEL": 16, "TIMEOUT": 32, "INTERNAL": 64}
 
 
@@ -87,6 +88,13 @@ _SIGS = {
                                          c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
     "qsa_sparse_attn_decode_noalloc": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p,
                                                   c_void_p, c_void_p, c_void_p, c_int32, c_void_p]),
+    "qsa_cp_shard_positions": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p,
+                                         c_void_p]),
+    "qsa_index_merge_candidates": (c_int32, [_S, _B, c_int32, c_void_p, c_void_p, c_void_p,
+                                             c_int32, c_int32, c_void_p, c_void_p, c_void_p,
+                                             c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qsa_attn_merge_partials": (c_int32, [c_int32, c_int32, c_int32, c_int32, c_void_p, c_void_p,
+                                          c_void_p, c_void_p, c_void_p]),
     "qsa_sparse_attn_backward": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                            c_void_p, c_void_p]),
@@ -175,6 +183,33 @@ def qsa_sparse_attn_decode_noalloc(cfg, batch, q, k_pool, v_pool, sel, n_sel, ou
                                                _p(k_pool), _p(v_pool), _p(sel), _p(n_sel), _p(out),
                                                _p(lse), int(num_splits), _stream(stream)),
            "qsa_sparse_attn_decode_noalloc")
+
+
+def qsa_cp_shard_positions(q_pos, num_q, shard_start, shard_len, pos_sel, pos_attn, stream=None):
+    _check(_lib.qsa_cp_shard_positions(_p(q_pos), int(num_q), int(shard_start), int(shard_len),
+                                       _p(pos_sel), _p(pos_attn), _stream(stream)),
+           "qsa_cp_shard_positions")
+
+
+def qsa_index_merge_candidates(cfg, batch, nparts, part_sel, part_scores, part_block_lo, block_lo,
+                               block_hi, sel, n_sel, sel_scores, local_sel, local_n, workspace,
+                               ws_bytes, stream=None):
+    """part_block_lo: a host sequence of nparts ints."""
+    lo = (c_int32 * int(nparts))(*[int(x) for x in part_block_lo])
+    _check(_lib.qsa_index_merge_candidates(ctypes.byref(cfg), ctypes.byref(batch), int(nparts),
+                                           _p(part_sel), _p(part_scores), ctypes.cast(lo, c_void_p),
+                                           int(block_lo), int(block_hi), _p(sel), _p(n_sel),
+                                           _p(sel_scores), _p(local_sel), _p(local_n),
+                                           _p(workspace), int(ws_bytes), _stream(stream)),
+           "qsa_index_merge_candidates")
+
+
+def qsa_attn_merge_partials(nparts, num_q, num_q_heads, head_dim, part_out, part_lse, out, lse=None,
+                            stream=None):
+    _check(_lib.qsa_attn_merge_partials(int(nparts), int(num_q), int(num_q_heads), int(head_dim),
+                                        _p(part_out), _p(part_lse), _p(out), _p(lse),
+                                        _stream(stream)),
+           "qsa_attn_merge_partials")
 
 
 def qsa_sparse_attn_backward(cfg, batch, q, k_pool, v_pool, sel, n_sel, out, lse, dout, dq,

@@ -103,6 +103,10 @@ qsa_status_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_batch_t* batc
     case QSA_OP_SPARSE_ATTN_DECODE:
       *bytes = qsa::sparse_decode_workspace_bytes(g, qsa::resolve_sparse_splits(g, num_splits));
       return QSA_OK;
+    case QSA_OP_MERGE_CANDIDATES:
+      if (num_splits < 1 || num_splits > qsa::kMaxCpParts) return QSA_ERR_INVALID_ARG;
+      *bytes = qsa::cp_merge_workspace_bytes(g, num_splits);
+      return QSA_OK;
     case QSA_OP_DENSE_ATTN_DECODE: {
       const int s = qsa::resolve_dense_splits(g, num_splits);
       *bytes = s > 1 ? qsa::dense_decode_workspace_bytes(g, s) : 0;
@@ -218,6 +222,52 @@ qsa_status_t qsa_sparse_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* 
     return QSA_ERR_WORKSPACE;
   return from_cuda(qsa::launch_sparse_attn(g, q, k_pool, v_pool, sel, n_sel, g.topk + 1, out,
                                            lse, s, workspace, (cudaStream_t)stream));
+}
+
+qsa_status_t qsa_cp_shard_positions(const int32_t* q_pos, int32_t num_q, int32_t shard_start,
+                                    int32_t shard_len, int32_t* pos_sel, int32_t* pos_attn,
+                                    qsa_stream_t stream) {
+  if (num_q < 0 || shard_start < 0 || shard_len < 64 || shard_start % 64 || shard_len % 64)
+    return QSA_ERR_INVALID_ARG;
+  if (num_q == 0) return QSA_OK;
+  if (!q_pos || !pos_sel || !pos_attn) return QSA_ERR_INVALID_ARG;
+  return from_cuda(qsa::launch_cp_positions(q_pos, num_q, shard_start, shard_len, pos_sel, pos_attn,
+                                            (cudaStream_t)stream));
+}
+
+qsa_status_t qsa_index_merge_candidates(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                                        int32_t nparts, const int32_t* part_sel,
+                                        const float* part_scores, const int32_t* part_block_lo,
+                                        int32_t block_lo, int32_t block_hi, int32_t* sel,
+                                        int32_t* n_sel, float* sel_scores, int32_t* local_sel,
+                                        int32_t* local_n, void* workspace, size_t ws_bytes,
+                                        qsa_stream_t stream) {
+  Geometry g;
+  qsa_status_t st = make_geometry(cfg, batch, &g, true);
+  if (st != QSA_OK) return st;
+  if (nparts < 1 || nparts > qsa::kMaxCpParts || !part_block_lo || block_lo < 0 || block_hi < block_lo)
+    return QSA_ERR_INVALID_ARG;
+  if (g.num_q == 0) return QSA_OK;
+  if (!part_sel || !part_scores || !sel || !n_sel || !local_sel || !local_n) return QSA_ERR_INVALID_ARG;
+  for (int p = 0; p < nparts; ++p)
+    if (part_block_lo[p] < 0) return QSA_ERR_INVALID_ARG;
+  const size_t need = qsa::cp_merge_workspace_bytes(g, nparts);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return QSA_ERR_WORKSPACE;
+  return from_cuda(qsa::launch_cp_merge(g, nparts, part_sel, part_scores, part_block_lo, block_lo,
+                                        block_hi, sel, n_sel, sel_scores, local_sel, local_n,
+                                        workspace, (cudaStream_t)stream));
+}
+
+qsa_status_t qsa_attn_merge_partials(int32_t nparts, int32_t num_q, int32_t num_q_heads,
+                                     int32_t head_dim, const void* part_out, const float* part_lse,
+                                     void* out, float* lse, qsa_stream_t stream) {
+  if (nparts < 1 || num_q < 0 || num_q_heads < 1 || (head_dim != 64 && head_dim != 128))
+    return QSA_ERR_INVALID_ARG;
+  if (num_q == 0) return QSA_OK;
+  if (!part_out || !part_lse || !out) return QSA_ERR_INVALID_ARG;
+  return from_cuda(qsa::launch_cp_merge_partials(nparts, num_q, num_q_heads, head_dim, part_out,
+                                                 part_lse, out, lse, (cudaStream_t)stream));
 }
 
 qsa_status_t qsa_sparse_attn_backward(const qsa_config_t* cfg, const qsa_batch_t* batch,

@@ -48,6 +48,18 @@ cudaError_t launch_dense_attn(const Geometry& g, const void* q, const void* k_po
                               const void* v_pool, void* out, float* lse, int splits, void* ws,
                               cudaStream_t s);
 
+// cp.cu (context parallel)
+constexpr int kMaxCpParts = 64;
+cudaError_t launch_cp_positions(const int32_t* q_pos, int num_q, int start, int len,
+                                int32_t* pos_sel, int32_t* pos_attn, cudaStream_t s);
+size_t cp_merge_workspace_bytes(const Geometry& g, int nparts);
+cudaError_t launch_cp_merge(const Geometry& g, int nparts, const int32_t* part_sel,
+                            const float* part_scores, const int32_t* part_lo, int lo, int hi,
+                            int32_t* sel, int32_t* n_sel, float* sel_scores, int32_t* local_sel,
+                            int32_t* local_n, void* ws, cudaStream_t s);
+cudaError_t launch_cp_merge_partials(int nparts, int num_q, int Hq, int D, const void* part_out,
+                                     const float* part_lse, void* out, float* lse, cudaStream_t s);
+
 // attn_bwd.cu
 cudaError_t launch_sparse_attn_bwd(const Geometry& g, const void* q, const void* k_pool,
                                    const void* v_pool, const int32_t* sel, const int32_t* n_sel,
