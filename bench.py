@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 METRIC = "QSA prefill tok/s and decode µs/step at 1M ctx; % of HBM/tensor roofline"
 PREFILL = "C4"
 DECODE = "C5"
+DISTILL = "DISTILL"
 
 
 # ------------------------------------------------------------------------------------ helpers
@@ -52,6 +53,15 @@ def load_peaks():
         return dict(hbm=float(d["hbm_gbs"]), tf=float(d["bf16_tflops"]),
                     tf_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
     return dict(hbm=6650.0, tf=1590.0, tf_sus=1400.0, src="fallback")
+
+
+def DISTILL_CONFIG():
+    """The distillation-signal workload: a 1,024-token chunk at 65,536 tokens of context with the
+    layer's heads (32q/4kv x 128, indexer 4 x 128)."""
+    from qsa_synth import Config
+
+    return Config("distill_chunk1024_ctx65536", "prefill", 1, 65536, 1024, 32, 4, 128, 4, 128,
+                  needles=64, shuffle_pages=True, seed=0x05A6)
 
 
 def positions_of(t: int, topk: int = 512) -> int:
@@ -174,7 +184,8 @@ class Workload:
         from qsa_synth.device import DeviceInputs
 
         self.torch = torch
-        self.c = c = CONFIGS[name] if not chunk else CONFIGS[name].replace(n_new=chunk)
+        base = CONFIGS[name] if name in CONFIGS else DISTILL_CONFIG()
+        self.c = c = base if not chunk else base.replace(n_new=chunk)
         self.di = d = DeviceInputs(c, integer=False, device=device)
         self.cfg = QsaConfig.make(c.Hq, c.Hkv, c.D, c.Di, topk=c.topk)
         self.runner = QsaRunner(self.cfg, device)
@@ -563,6 +574,72 @@ def oracle_decode_baseline():
                        f"{c.ctx}-token context; the step is extrapolated as {c.batch} x that")
 
 
+# ------------------------------------------------------------------------------------ training
+
+def _time_ms(torch, fn, reps: int) -> float:
+    fn()
+    torch.cuda.synchronize()
+    ev = []
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+
+def training_kernels(w: Workload, peaks, reps: int = 3):
+    """The training-side kernels on the prefill workload's device inputs: the sparse attention
+    backward (16,384 rows at 1M context, gradients accumulated into fp32 cache-shaped pools), and
+    the indexer-distillation signal on a 1,024-row chunk at 65,536 tokens of context (dense work:
+    two q.k passes over each row's whole context)."""
+    import numpy as np
+
+    torch = w.torch
+    from learned_block_sparse_qsa_b200 import qsa_index_distill_kl, qsa_sparse_attn_backward
+
+    c, d, r, b = w.c, w.di, w.runner, w.b
+    lse = torch.empty(c.num_q, c.Hq, dtype=torch.float32, device=d.q.device)
+    w.step(False)
+    from learned_block_sparse_qsa_b200 import qsa_sparse_attn_prefill
+
+    qsa_sparse_attn_prefill(w.cfg, b, d.q, d.k_pool, d.v_pool, w.sel, w.n_sel, w.out, lse)
+    dout = torch.randn(d.q.shape, device=d.q.device, generator=torch.Generator(device=d.q.device).manual_seed(1)).to(torch.bfloat16)
+    dq = torch.empty(d.q.shape, dtype=torch.float32, device=d.q.device)
+    dk = torch.zeros(d.k_pool.shape, dtype=torch.float32, device=d.q.device)
+    dv = torch.zeros_like(dk)
+    bwd_ms = _time_ms(torch, lambda: qsa_sparse_attn_backward(
+        w.cfg, b, d.q, d.k_pool, d.v_pool, w.sel, w.n_sel, w.out, lse, dout, dq, dk, dv), reps)
+    work = algorithmic(c, w.q_pos_host)
+    bwd_flops = work["attn_flops"] * 2.5  # S, dA, dQ, dK, dV products: 5 of the forward's 2
+    del dk, dv, dq, dout
+    torch.cuda.empty_cache()
+
+    wd = Workload(DISTILL, d.q.device)
+    cd = wd.c
+    kl = torch.empty(cd.num_q, dtype=torch.float32, device=d.q.device)
+    dd = wd.di
+    wd.step(False)  # compresses the chunk's keys
+    dist_ms = _time_ms(torch, lambda: qsa_index_distill_kl(
+        wd.cfg, wd.b, dd.q, dd.k_pool, dd.idx_q, dd.idx_w, dd.kcomp_pool, kl), reps)
+    t = np.asarray(wd.q_pos_host, dtype=np.int64)
+    dist_flops = int((2 * cd.Hq * cd.D * (t + 1 + 4 * (t // 4))).sum() + (2 * 4 * cd.Di * (t // 4)).sum())
+    del wd
+    torch.cuda.empty_cache()
+    return {
+        "sparse_attn_backward": {"workload": c.name, "ms": bwd_ms, "tokens_per_s": c.num_q / (bwd_ms * 1e-3),
+                                 "gathered_gbs": work["attn_bytes"] / (bwd_ms * 1e-3) / 1e9,
+                                 "tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,
+                                 "note": "dk/dv added to fp32 pools by vector atomics"},
+        "distill_kl": {"workload": cd.name, "ms": dist_ms, "tflops": dist_flops / (dist_ms * 1e-3) / 1e12,
+                       "peak_tflops": peaks["tf"], "frac": dist_flops / (dist_ms * 1e-3) / 1e12 / peaks["tf"],
+                       "kernel": "mma.sync"},
+    }
+
+
 # ------------------------------------------------------------------------------------ main
 
 def main():
@@ -671,6 +748,8 @@ def main():
     log(f"prefill e2e {e2e_ms:.3f} ms/step")
     dense_ms = dense_time_ms(w, False, 3)
     log(f"dense prefill {dense_ms:.1f} ms ({work['dense_flops'] / (dense_ms * 1e-3) / 1e12:.1f} TFLOP/s)")
+    train = training_kernels(w, peaks)
+    log("training kernels: " + json.dumps(train))
     del w
     torch.cuda.empty_cache()
 
@@ -734,6 +813,7 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},
+            "training_kernels": train,
             "dense_baseline": {"prefill_ms": dense_ms, "sparse_over_dense_speedup": dense_ms / ms_step,
                                "dense_prefill_tflops": work["dense_flops"] / (dense_ms * 1e-3) / 1e12,
                                "decode_us": dense_dec_ms * 1000,
