@@ -72,7 +72,8 @@ typedef enum qsa_op {
   QSA_OP_INDEX_SCORE_TOPK = 1,
   QSA_OP_SPARSE_ATTN_DECODE = 2,
   QSA_OP_DENSE_ATTN_DECODE = 3,
-  QSA_OP_MERGE_CANDIDATES = 4 /* num_splits = number of parts */
+  QSA_OP_MERGE_CANDIDATES = 4, /* num_splits = number of parts */
+  QSA_OP_DECODE_STEP = 5       /* num_splits as passed to qsa_decode_step */
 } qsa_op_t;
 
 typedef struct qsa_config {
@@ -182,6 +183,25 @@ qsa_status_t qsa_sparse_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* 
                                     const int32_t* sel, const int32_t* n_sel, void* out,
                                     float* lse, int32_t num_splits, void* workspace,
                                     size_t ws_bytes, qsa_stream_t stream);
+
+/* The whole decode step in ONE launch (section "Three speed claims, three different experiments":
+ * decode with batch 4 and three extra multi-token-prediction positions): compress the step's new
+ * keys (as qsa_index_compress; n_new may be 0), select for every row (as qsa_index_score_topk),
+ * and attend split-K (as qsa_sparse_attn_decode), in one cooperative kernel of one CTA per SM
+ * whose CTAs wait for one another only on the data they need (bounded waits, ~1 s, then
+ * QSA_DEVERR_TIMEOUT).  Results equal the three calls'.  Decode-sized batches: idx_dim 128,
+ * Hq/Hkv <= 8, num_q <= 256 (QSA_ERR_UNSUPPORTED otherwise, or when the driver has no tensor-map
+ * encoder).  workspace: qsa_workspace_size(..., QSA_OP_DECODE_STEP, num_splits, ...) bytes,
+ * ZERO-FILLED before its first use: it holds the launch's synchronisation words, which every
+ * completed call leaves at zero again (after a call that reported QSA_DEVERR_TIMEOUT, zero it
+ * again).  Calls sharing a workspace must not overlap on the GPU. */
+qsa_status_t qsa_decode_step(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                             const void* idx_k_new, const int32_t* new_seq, const int32_t* new_pos,
+                             int32_t n_new, void* kcomp_pool, const void* idx_q, const void* idx_w,
+                             const void* q, const void* k_pool, const void* v_pool, int32_t* sel,
+                             int32_t* n_sel, float* sel_scores, void* out, float* lse,
+                             int32_t num_splits, void* workspace, size_t ws_bytes,
+                             qsa_stream_t stream);
 
 /* No counterpart in the article: a variant of qsa_sparse_attn_decode for callers that cannot
  * allocate device memory at step time (for example a serving engine whose memory planner owns all

@@ -24,7 +24,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA = 0, 1, 2, 3, 4
 QSA_OP_INDEX_SCORE_TOPK, QSA_OP_SPARSE_ATTN_DECODE, QSA_OP_DENSE_ATTN_DECODE = 1, 2, 3
-QSA_OP_MERGE_CANDIDATES = 4
+QSA_OP_MERGE_CANDIDATES, QSA_OP_DECODE_STEP = 4, 5
 DEVERR = {"SEQ": 1, "POS": 2, "PAGE": 4, "GROUP": 8, "SEL": 16, "TIMEOUT": 32, "INTERNAL": 64}
 
 
@@ -88,6 +88,10 @@ _SIGS = {
                                          c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
     "qsa_sparse_attn_decode_noalloc": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p,
                                                   c_void_p, c_void_p, c_void_p, c_int32, c_void_p]),
+    "qsa_decode_step": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                  c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_size_t,
+                                  c_void_p]),
     "qsa_cp_shard_positions": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p,
                                          c_void_p]),
     "qsa_index_merge_candidates": (c_int32, [_S, _B, c_int32, c_void_p, c_void_p, c_void_p,
@@ -183,6 +187,18 @@ def qsa_sparse_attn_decode_noalloc(cfg, batch, q, k_pool, v_pool, sel, n_sel, ou
                                                _p(k_pool), _p(v_pool), _p(sel), _p(n_sel), _p(out),
                                                _p(lse), int(num_splits), _stream(stream)),
            "qsa_sparse_attn_decode_noalloc")
+
+
+def qsa_decode_step(cfg, batch, idx_k_new, new_seq, new_pos, n_new, kcomp_pool, idx_q, idx_w, q,
+                    k_pool, v_pool, sel, n_sel, sel_scores, out, lse, num_splits, workspace,
+                    ws_bytes, stream=None):
+    """The fused one-launch decode step (workspace zero-filled before its first use)."""
+    _check(_lib.qsa_decode_step(ctypes.byref(cfg), ctypes.byref(batch), _p(idx_k_new), _p(new_seq),
+                                _p(new_pos), int(n_new), _p(kcomp_pool), _p(idx_q), _p(idx_w),
+                                _p(q), _p(k_pool), _p(v_pool), _p(sel), _p(n_sel), _p(sel_scores),
+                                _p(out), _p(lse), int(num_splits), _p(workspace), int(ws_bytes),
+                                _stream(stream)),
+           "qsa_decode_step")
 
 
 def qsa_cp_shard_positions(q_pos, num_q, shard_start, shard_len, pos_sel, pos_attn, stream=None):

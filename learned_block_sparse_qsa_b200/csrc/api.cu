@@ -103,6 +103,11 @@ qsa_status_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_batch_t* batc
     case QSA_OP_SPARSE_ATTN_DECODE:
       *bytes = qsa::sparse_decode_workspace_bytes(g, qsa::resolve_sparse_splits(g, num_splits));
       return QSA_OK;
+    case QSA_OP_DECODE_STEP:
+      if (num_splits < 0) return QSA_ERR_INVALID_ARG;
+      if (!qsa::decode_step_supported(g)) return QSA_ERR_UNSUPPORTED;
+      *bytes = qsa::decode_step_workspace_bytes(g, num_splits);
+      return QSA_OK;
     case QSA_OP_MERGE_CANDIDATES:
       if (num_splits < 1 || num_splits > qsa::kMaxCpParts) return QSA_ERR_INVALID_ARG;
       *bytes = qsa::cp_merge_workspace_bytes(g, num_splits);
@@ -222,6 +227,31 @@ qsa_status_t qsa_sparse_attn_decode(const qsa_config_t* cfg, const qsa_batch_t* 
     return QSA_ERR_WORKSPACE;
   return from_cuda(qsa::launch_sparse_attn(g, q, k_pool, v_pool, sel, n_sel, g.topk + 1, out,
                                            lse, s, workspace, (cudaStream_t)stream));
+}
+
+qsa_status_t qsa_decode_step(const qsa_config_t* cfg, const qsa_batch_t* batch,
+                             const void* idx_k_new, const int32_t* new_seq, const int32_t* new_pos,
+                             int32_t n_new, void* kcomp_pool, const void* idx_q, const void* idx_w,
+                             const void* q, const void* k_pool, const void* v_pool, int32_t* sel,
+                             int32_t* n_sel, float* sel_scores, void* out, float* lse,
+                             int32_t num_splits, void* workspace, size_t ws_bytes,
+                             qsa_stream_t stream) {
+  Geometry g;
+  qsa_status_t st = sparse_common(cfg, batch, q, k_pool, v_pool, sel, n_sel, out, &g);
+  if (st != QSA_OK || g.num_q == 0) return st;
+  if (num_splits < 0 || n_new < 0 || n_new % 4 != 0) return QSA_ERR_INVALID_ARG;
+  if (!idx_q || !idx_w || !kcomp_pool || (n_new > 0 && (!idx_k_new || !new_seq || !new_pos)))
+    return QSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx_q) | reinterpret_cast<uintptr_t>(kcomp_pool) |
+       reinterpret_cast<uintptr_t>(idx_k_new)) & 15)
+    return QSA_ERR_INVALID_ARG;
+  if (!qsa::decode_step_supported(g) || qsa::tmap_encode_fn_available() == 0) return QSA_ERR_UNSUPPORTED;
+  const size_t need = qsa::decode_step_workspace_bytes(g, num_splits);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return QSA_ERR_WORKSPACE;
+  return from_cuda(qsa::launch_decode_step(g, idx_k_new, new_seq, new_pos, n_new, kcomp_pool, idx_q,
+                                           idx_w, q, k_pool, v_pool, sel, n_sel, sel_scores, out,
+                                           lse, num_splits, workspace, (cudaStream_t)stream));
 }
 
 qsa_status_t qsa_cp_shard_positions(const int32_t* q_pos, int32_t num_q, int32_t shard_start,

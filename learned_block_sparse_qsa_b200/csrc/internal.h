@@ -26,12 +26,22 @@ cudaError_t launch_compress(const Geometry& g, const void* idx_k, const int32_t*
 size_t score_workspace_bytes(const Geometry& g, int path);
 int resolve_score_path(const Geometry& g, int requested);
 bool score_path_runnable(const Geometry& g, int path);  // false: the driver lacks what it needs
+int tmap_encode_fn_available();
 bool score_redo_offset(const Geometry& g, int path, size_t* off);
 cudaError_t launch_score_topk(const Geometry& g, int path, const void* idx_q, const void* idx_w,
                               const void* kcomp, int32_t* sel, int32_t* n_sel, float* sel_scores,
                               void* ws, size_t ws_bytes, cudaStream_t s);
 cudaError_t launch_scores_only(const Geometry& g, const void* idx_q, const void* idx_w,
                                const void* kcomp, float* scores, int64_t ld, cudaStream_t s);
+
+// score_dec.cu: the fused decode step (one cooperative launch)
+bool decode_step_supported(const Geometry& g);
+size_t decode_step_workspace_bytes(const Geometry& g, int num_splits);
+cudaError_t launch_decode_step(const Geometry& g, const void* idx_k_new, const int32_t* new_seq,
+                               const int32_t* new_pos, int n_new, void* kcomp, const void* idx_q,
+                               const void* idx_w, const void* q, const void* k_pool,
+                               const void* v_pool, int32_t* sel, int32_t* n_sel, float* sel_scores,
+                               void* out, float* lse, int num_splits, void* ws, cudaStream_t s);
 
 // attn.cu
 int resolve_sparse_splits(const Geometry& g, int requested);

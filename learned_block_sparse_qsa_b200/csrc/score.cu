@@ -720,6 +720,8 @@ int resolve_score_path(const Geometry& g, int requested) {
 // maps.  Without the driver's encoder they cannot run, and a silent switch to the mma.sync
 // streaming kernel would be a large, invisible slowdown: the call reports it instead (path 4
 // asks for the streaming kernel explicitly).
+int tmap_encode_fn_available() { return tmap_encode_fn() != nullptr; }
+
 bool score_path_runnable(const Geometry& g, int path) {
   const bool needs_tma = (path == 1 && g.Di == 128) || path == 3;
   return !needs_tma || tmap_encode_fn() != nullptr;

@@ -30,6 +30,7 @@
 #include "internal.h"
 #include "score_common.cuh"
 #include "select.cuh"
+#include "attn_sw.cuh"
 
 namespace qsa {
 namespace {
@@ -53,15 +54,17 @@ static_assert(DM_THREADS == 512 && 2 * DM_THREADS >= DS_MAXW,
 static_assert(DS_MAXW / DS_WARPS * DS_KC <= DM_MAXU && (DS_CTA_MERGE_W - 1) * DS_KW <= DM_MAXU,
               "union bound");
 
-struct DecSmem {
-  static constexpr int STAGES = DS_WARPS * DS_NST * DS_PAGE;  // first, 1024-byte aligned
-  static constexpr int BUF = DS_WARPS * 4 * DS_CAP * 8;
-  static constexpr int MLIST = DS_WARPS * 4 * DS_KW * 8;      // warp lists for the CTA merge
-  static constexpr int MBOUND = DS_WARPS * 4 * 8;
-  static constexpr int PID = DS_WARPS * DS_MAXPG * 4;
-  static constexpr int BAR = DS_WARPS * DS_NST * 8;
+template <int NW>
+struct DecSmemT {
+  static constexpr int STAGES = NW * DS_NST * DS_PAGE;  // first, 1024-byte aligned
+  static constexpr int BUF = NW * 4 * DS_CAP * 8;
+  static constexpr int MLIST = NW * 4 * DS_KW * 8;      // warp lists for the CTA merge
+  static constexpr int MBOUND = NW * 4 * 8;
+  static constexpr int PID = NW * DS_MAXPG * 4;
+  static constexpr int BAR = NW * DS_NST * 8;
   static constexpr int TOTAL = STAGES + BUF + MLIST + MBOUND + PID + BAR + 1024;  // + alignment
 };
+using DecSmem = DecSmemT<DS_WARPS>;
 static_assert(DS_CTAS * (DecSmem::TOTAL + 1024) <= 233472, "resident CTAs per SM");
 
 struct DecPlan {
@@ -77,24 +80,28 @@ __host__ __device__ inline int pad2(int n) { return (n + 1) & ~1; }
 // Chunking of the candidate pages: one warp per chunk, DS_CTAS CTAs per SM in total, at least
 // DS_MINW chunks per tile (a row's union then holds >= 2,048 keys whenever any list dropped
 // keys), chunks of at most DS_MAXPG pages.
-bool dec_plan(const Geometry& g, DecPlan* p) {
+// nw: warps per CTA; resident_warps: warps the GPU runs at once (all of them stream together).
+bool dec_plan_nw(const Geometry& g, int nw, long long resident_warps, DecPlan* p) {
   p->T = (g.num_q + 3) / 4;
   const long long pages = ((long long)g.max_pos / 4 + 15) / 16;  // candidates are b < t/4
   const long long P = pages > 0 ? pages : 1;
-  long long W = ((long long)DS_CTAS * num_sms() * DS_WARPS + p->T - 1) / p->T;
+  long long W = (resident_warps + p->T - 1) / p->T;
   W = W < DS_MINW ? DS_MINW : (W > DS_MAXW ? DS_MAXW : W);
   if (W > P) W = P;
   long long chunk = (P + W - 1) / W;
   if (chunk > DS_MAXPG) chunk = DS_MAXPG;
   W = (P + chunk - 1) / chunk;
-  W = (W + DS_WARPS - 1) / DS_WARPS * DS_WARPS;  // trailing chunks may be empty
+  W = (W + nw - 1) / nw * nw;  // trailing chunks may be empty
   if (W > DS_MAXW) return false;
   p->W = (int)W;
   p->chunk = (int)chunk;
   const bool merge = W >= DS_CTA_MERGE_W;
-  p->nl = merge ? p->W / DS_WARPS : p->W;
+  p->nl = merge ? p->W / nw : p->W;
   p->lk = merge ? DS_KC : DS_KW;
   return true;
+}
+bool dec_plan(const Geometry& g, DecPlan* p) {
+  return dec_plan_nw(g, DS_WARPS, (long long)DS_CTAS * num_sms() * DS_WARPS, p);
 }
 
 // Per query row, its nl lists are contiguous so that the merge fetches the row's union with one
@@ -172,25 +179,38 @@ __device__ __forceinline__ u64 warp_fold_two16(u64 top, u64 v) {
   return v;
 }
 
-__global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
-    dec_score_kernel(ScoreArgs a, const __grid_constant__ CUtensorMap tmK, DecWs ws, int W, int chunk,
-                     int nl) {
-  extern __shared__ uint8_t smem_raw[];
+// Optional wait of the warps whose pages hold blocks compressed earlier in the same launch (the
+// fused decode step): they wait for `*ctr >= target` before streaming those pages.
+struct NewBlockWait {
+  const int* ctr = nullptr;
+  int target = 0;
+  const int32_t* new_seq = nullptr;
+  const int32_t* new_pos = nullptr;
+  int n_groups = 0;
+};
+
+// The streaming part of the decode indexer for virtual CTA `vblock` of NW warps (all threads of
+// the calling block take part).  smem_raw: DecSmemT<NW>::TOTAL bytes.
+template <int NW>
+__device__ __forceinline__ void dec_score_body(const ScoreArgs& a, const CUtensorMap* tmK, const DecWs& ws,
+                                               int W, int chunk, int nl, int vblock, uint8_t* smem_raw,
+                                               const NewBlockWait& nbw) {
+  using DecSmem = DecSmemT<NW>;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * DS_WARPS + warp;
+  const int gw = vblock * NW + warp;
   const int T = (a.num_q + 3) / 4;
   const int tile = gw / W, wc = gw % W;
-  if (tile >= T) return;  // the whole CTA (W is a multiple of DS_WARPS)
+  if (tile >= T) return;  // the whole CTA (W is a multiple of NW)
   const bool cta_merge = nl != W;
 
   const uint32_t stage0 = smem_addr(smem) + warp * (DS_NST * DS_PAGE);
   u64* buf = reinterpret_cast<u64*>(smem + DecSmem::STAGES) + warp * 4 * DS_CAP;
   u64* mlist = reinterpret_cast<u64*>(smem + DecSmem::STAGES + DecSmem::BUF);  // [warp][row][16]
-  u64* mbound = mlist + DS_WARPS * 4 * DS_KW;                                  // [warp][row]
-  int* pid = reinterpret_cast<int*>(mbound + DS_WARPS * 4) + warp * DS_MAXPG;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<int*>(mbound + DS_WARPS * 4) +
-                                              DS_WARPS * DS_MAXPG) + warp * DS_NST;
+  u64* mbound = mlist + NW * 4 * DS_KW;                                  // [warp][row]
+  int* pid = reinterpret_cast<int*>(mbound + NW * 4) + warp * DS_MAXPG;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<int*>(mbound + NW * 4) +
+                                              NW * DS_MAXPG) + warp * DS_NST;
   if (lane == 0) {
     for (int s = 0; s < DS_NST; ++s) mbar_init(&bar[s], 1);
     mbar_fence_init();
@@ -269,6 +289,25 @@ __global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
       }
       pid[i] = pg;
     }
+    if (nbw.ctr && lane == 0) {  // pages holding blocks compressed earlier in this launch
+      bool hit = false;
+      for (int j = 0; j < nbw.n_groups && !hit; ++j) {
+        const int bp = nbw.new_pos[4 * j] / 64;
+        hit = nbw.new_seq[4 * j] == seg && bp >= p0 && bp < p0 + np;
+      }
+      if (hit) {
+        const volatile int* c = nbw.ctr;
+        const long long t0 = clock64();
+        while (*c < nbw.target) {
+          if (clock64() - t0 > kWaitLimitCycles) {
+            flag_error(a.err, QSA_DEVERR_TIMEOUT);
+            break;
+          }
+        }
+        __threadfence();
+        asm volatile("fence.proxy.async.global;\n" ::: "memory");
+      }
+    }
     __syncwarp();
     auto issue = [&](int i) {  // lane 0 only
       const int s = (base + i) % DS_NST;
@@ -278,8 +317,8 @@ __global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         mbar_arrive_expect_tx(&bar[s], DS_PAGE);
         const uint64_t pol = l2_evict_first_policy();
-        tma2d_hint(stage0 + s * DS_PAGE, &tmK, 0, pg * 16, &bar[s], pol);
-        tma2d_hint(stage0 + s * DS_PAGE + DS_PAGE / 2, &tmK, 64, pg * 16, &bar[s], pol);
+        tma2d_hint(stage0 + s * DS_PAGE, tmK, 0, pg * 16, &bar[s], pol);
+        tma2d_hint(stage0 + s * DS_PAGE + DS_PAGE / 2, tmK, 64, pg * 16, &bar[s], pol);
       } else {
         mbar_arrive(&bar[s]);  // no data: the page's blocks are masked below
       }
@@ -406,24 +445,31 @@ __global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
   }
 
   if (!cta_merge) return;
-  // CTA merge: warp r (< 4) folds the DS_WARPS lists of row r into one list of DS_KC keys
+  // CTA merge: warp r (< 4) folds the NW lists of row r into one list of DS_KC keys
   __syncthreads();
   const int r = warp;
   if (r >= 4 || tile * 4 + r >= a.num_q) return;
   u64 top = 0, bound = 0;
   int nz = 0;
-  for (int w = 0; w < DS_WARPS; w += 2) {
+  for (int w = 0; w < NW; w += 2) {
     const u64 v = mlist[((w + (lane >> 4)) * 4 + r) * DS_KW + (lane & 15)];
     nz += __popc(__ballot_sync(0xffffffffu, v != 0ull));
     top = warp_fold_two16(top, v);
   }
-  for (int w = 0; w < DS_WARPS; ++w) bound = mbound[w * 4 + r] > bound ? mbound[w * 4 + r] : bound;
+  for (int w = 0; w < NW; ++w) bound = mbound[w * 4 + r] > bound ? mbound[w * 4 + r] : bound;
   const u64 kth = __shfl_sync(0xffffffffu, top, 31);
   if (nz > DS_KC && kth > bound) bound = kth;  // the CTA merge itself dropped keys below kth
   const long long row = (long long)tile * 4 + r;
-  const int cidx = wc / DS_WARPS;
+  const int cidx = wc / NW;
   ws.lists[(row * nl + cidx) * DS_KC + lane] = top;
   if (lane == 0) ws.bounds[row * pad2(nl) + cidx] = bound;
+}
+
+__global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
+    dec_score_kernel(ScoreArgs a, const __grid_constant__ CUtensorMap tmK, DecWs ws, int W, int chunk,
+                     int nl) {
+  extern __shared__ uint8_t smem_raw[];
+  dec_score_body<DS_WARPS>(a, &tmK, ws, W, chunk, nl, blockIdx.x, smem_raw, NewBlockWait{});
 }
 
 // ------------------------------------------------------------------ merge (one CTA per row)
@@ -571,9 +617,10 @@ __device__ u64 cta_kth_largest(const u64* keys, int n, int need, uint32_t* hist,
 // One CTA per query row.  The row's lists come in block order (list l covers a block range below
 // list l+1's) and each is sorted by key, so the need keys >= tau are a prefix of every list: the
 // output is the lists' prefixes in list order, each put in block order by a warp-level rank.
-__global__ void __launch_bounds__(DM_THREADS)
-    dec_merge_kernel(ScoreArgs a, DecWs ws, int nl, int lk) {
-  extern __shared__ __align__(128) uint8_t smem[];
+// The merge of query row `row` by all DM_THREADS threads of the calling block; smem:
+// MergeSmem::TOTAL bytes, 128-byte aligned.  A row it cannot settle gets ws.redo[row] = 1.
+__device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& ws, int nl, int lk,
+                                               const int row, uint8_t* smem) {
   u64* keys = reinterpret_cast<u64*>(smem);
   u64* bnds = reinterpret_cast<u64*>(smem + MergeSmem::KEYS);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + MergeSmem::KEYS + MergeSmem::BOUNDS);
@@ -589,8 +636,13 @@ __global__ void __launch_bounds__(DM_THREADS)
   uint32_t* sel3 = reinterpret_cast<uint32_t*>(tail + 520);  // digit, above, count, n in bin
   u64* s_tau = reinterpret_cast<u64*>(tail + 536);
 
-  const int row = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int NW = DM_THREADS / 32;
+  if (tid == 0) {  // initialised on every path, so that a caller can invalidate it afterwards
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
   const int seq = a.q_seq[row], pos = a.q_pos[row];
   const bool ok = seq >= 0 && seq < a.batch && pos >= 0 && pos / 64 < a.max_pages && pos <= a.max_pos;
   if (!ok) {  // already flagged by the score kernel
@@ -618,11 +670,6 @@ __global__ void __launch_bounds__(DM_THREADS)
   // the row's nl lists (zero-padded) and their bounds, one bulk copy each
   const int nlp = pad2(nl);
   const int U = nl * lk;
-  if (tid == 0) {
-    mbar_init(bar, 1);
-    mbar_fence_init();
-  }
-  __syncthreads();
   if (tid == 0) {
     mbar_arrive_expect_tx(bar, (uint32_t)(U * 8 + nlp * 8));
     bulk_g2s(smem_addr(keys), ws.lists + (long long)row * U, (uint32_t)(U * 8), bar);
@@ -789,6 +836,264 @@ __global__ void __launch_bounds__(DM_THREADS)
   }
 }
 
+__global__ void __launch_bounds__(DM_THREADS) dec_merge_kernel(ScoreArgs a, DecWs ws, int nl, int lk) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  dec_merge_body(a, ws, nl, lk, blockIdx.x, smem);
+}
+
+// ------------------------------------------------------------------ exact path for one row
+// The row's every candidate score on CUDA cores (4 heads x 128 dims per block), as 64-bit keys in
+// `keys` (global, >= t/4 entries), then the CTA radix select and a block-order sort.  For rows the
+// split lists cannot settle (adversarial score orders): about a millisecond per 1M-token row.
+struct ExactSmem {
+  static constexpr int Q = 4 * 128 * 4;  // queries as fp32
+  static constexpr int W = 16;
+  static constexpr int HIST = 2048 * 4;
+  static constexpr int RED = 48 * 8;
+  static constexpr int WSUM = 32 * 4;
+  static constexpr int SEL3 = 16;
+  static constexpr int BLK = 512 * 4;
+  static constexpr int SC = 512 * 4;
+  static constexpr int TOTAL = Q + W + HIST + RED + WSUM + SEL3 + BLK + SC + 16;
+};
+
+__device__ __forceinline__ void exact_row_body(const ScoreArgs& a, const int row, u64* keys, uint8_t* smem) {
+  float* sq = reinterpret_cast<float*>(smem);
+  float* sw = sq + 4 * 128;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + ExactSmem::Q + ExactSmem::W);
+  u64* red = reinterpret_cast<u64*>(smem + ExactSmem::Q + ExactSmem::W + ExactSmem::HIST);
+  uint32_t* wsum = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(red) + ExactSmem::RED);
+  uint32_t* sel3 = wsum + 32;
+  uint32_t* sblk = sel3 + 4;
+  float* ssc = reinterpret_cast<float*>(sblk + 512);
+  int* cnt = reinterpret_cast<int*>(ssc + 512);
+  const int tid = threadIdx.x;
+  const int seq = a.q_seq[row], pos = a.q_pos[row];
+  const int lim = pos / 4;
+  const int need = min(a.topk, lim);
+  for (int i = tid; i < 4 * 128; i += DM_THREADS)
+    sq[i] = __bfloat162float(a.idx_q[(long long)row * 4 * 128 + i]);
+  if (tid < 4) sw[tid] = __bfloat162float(a.idx_w[(long long)row * 4 + tid]);
+  if (tid == 0) *cnt = 0;
+  __syncthreads();
+  const int32_t* pt = a.page_table + (long long)seq * a.max_pages;
+  for (int b = tid; b < lim; b += DM_THREADS) {
+    const int page = pt[b >> 4];
+    float sc = 0.f;
+    if (page >= 0 && page < a.num_pages) {
+      const uint4* k4 = reinterpret_cast<const uint4*>(a.kcomp + ((long long)page * 16 + (b & 15)) * 128);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int c = 0; c < 16; ++c) {
+        const uint4 v = k4[c];
+        const bf16* kh = reinterpret_cast<const bf16*>(&v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float kd = __bfloat162float(kh[e]);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) acc[h] = fmaf(sq[h * 128 + c * 8 + e], kd, acc[h]);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 4; ++h) sc = fmaf(sw[h], fmaxf(acc[h], 0.f), sc);
+    } else {
+      flag_error(a.err, QSA_DEVERR_PAGE);
+    }
+    keys[b] = make_key(sc, (uint32_t)b);
+  }
+  __syncthreads();
+  const u64 kth = need > 0 ? cta_kth_largest(keys, lim, need, hist, red, wsum, sel3) : ~0ull;
+  for (int b = tid; b < lim; b += DM_THREADS) {
+    const u64 k = keys[b];
+    if (need > 0 && k >= kth) {
+      const int i = atomicAdd(cnt, 1);
+      if (i < 512) {
+        sblk[i] = (uint32_t)b;
+        ssc[i] = key_score(k);
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const int n = min(*cnt, need);
+    if (n > 0) warp_sort_blocks(sblk, ssc, n);
+    __syncwarp();
+    write_selection(row, n, lim, sblk, ssc, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ the fused decode step
+// One cooperative launch, one CTA of 512 threads per SM, for a decode-sized batch:
+//   compress   the step's new blocks (one 4-key group per CTA, first CTAs);
+//   score      16 warps per CTA stream the compressed keys as dec_score_kernel does (warps whose
+//              pages hold a block compressed in this launch wait for it first);
+//   merge      CTA r selects row r exactly (dec_merge_body) once every CTA of its 4-row tile has
+//              posted its lists, or, for a row the lists cannot settle, by the exact path;
+//   attend     CTA i runs split i % S of row i / S once that row is selected (the swap-AB kernel
+//              body; the last split of a row merges the partials);
+// with no grid-wide barrier: each CTA waits (bounded, ~1 s) only on the counters or flags of the
+// work it needs, in workspace words that are zero before the first call and that the last CTA to
+// leave sets back to zero.
+constexpr int FS_WARPS = 16;
+constexpr int FS_THREADS = FS_WARPS * 32;
+static_assert(FS_THREADS == DM_THREADS, "the merge body runs on the whole fused CTA");
+
+struct StepSync {
+  int* comp_done;   // [1] compressed groups
+  int* tile_done;   // [T] score CTAs finished per 4-row tile
+  int* merged;      // [num_q] row selected
+  int* exit_count;  // [1] CTAs that left
+};
+
+struct StepArgs {
+  ScoreArgs sa;
+  AttnArgs aa;
+  DecWs ws;
+  int W, chunk, nl, lk, T;
+  const bf16* idx_k_new;
+  const int32_t* new_seq;
+  const int32_t* new_pos;
+  int n_groups;
+  bf16* kcomp_w;
+  u64* exact_keys;
+  long long exact_ld;
+  StepSync sync;
+};
+
+__device__ __forceinline__ void inval_mbar(uint8_t* p) {
+  asm volatile("mbarrier.inval.shared::cta.b64 [%0];\n" ::"r"(smem_addr(p)) : "memory");
+}
+
+// Bounded wait (thread 0) for *w >= target; then acquire and make generic-proxy writes visible to
+// the async proxy.  Gives up after the wait limit with QSA_DEVERR_TIMEOUT.
+__device__ __forceinline__ void wait_geq(const int* w, int target, int32_t* err) {
+  const volatile int* v = w;
+  if (*v < target) {
+    const long long t0 = clock64();
+    while (*v < target) {
+      if (clock64() - t0 > kWaitLimitCycles) {
+        flag_error(err, QSA_DEVERR_TIMEOUT);
+        break;
+      }
+    }
+  }
+  __threadfence();
+  asm volatile("fence.proxy.async.global;\n" ::: "memory");
+}
+
+template <int D, int HKV, int SLC>
+__global__ void __launch_bounds__(FS_THREADS, 1)
+    decode_step_kernel(StepArgs p, const __grid_constant__ CUtensorMap tmK) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  using AC = SwCfg<D, HKV, SLC>;
+  const int tid = threadIdx.x;
+  const ScoreArgs& a = p.sa;
+
+  // ---- compress: group g (4 raw keys of one block) by 16 threads of CTA g % gridDim.x
+  int mine = 0;
+  for (int g = blockIdx.x; g < p.n_groups; g += gridDim.x) {
+    ++mine;
+    if (tid < 16) {
+      const long long r0 = (long long)g * 4;
+      const int seq = p.new_seq[r0], pos0 = p.new_pos[r0];
+      bool ok = pos0 >= 0 && pos0 % 4 == 0 && seq >= 0 && seq < a.batch && pos0 / 64 < a.max_pages;
+#pragma unroll
+      for (int i = 1; i < 4; ++i) ok = ok && p.new_seq[r0 + i] == seq && p.new_pos[r0 + i] == pos0 + i;
+      const int page = ok ? a.page_table[(long long)seq * a.max_pages + pos0 / 64] : -1;
+      if (ok && page >= 0 && page < a.num_pages) {
+        double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = reinterpret_cast<const uint4*>(p.idx_k_new + (r0 + i) * 128)[tid];
+          const bf16* h = reinterpret_cast<const bf16*>(&v);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] += (double)__bfloat162float(h[e]);
+        }
+        uint4 o;
+        bf16* oh = reinterpret_cast<bf16*>(&o);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) oh[e] = __double2bfloat16(acc[e] * 0.25);
+        reinterpret_cast<uint4*>(p.kcomp_w + ((long long)page * 16 + (pos0 / 4) % 16) * 128)[tid] = o;
+      } else if (tid == 0) {
+        flag_error(a.err, ok ? QSA_DEVERR_PAGE : QSA_DEVERR_GROUP);
+      }
+    }
+  }
+  if (mine) {
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      asm volatile("fence.proxy.async.global;\n" ::: "memory");
+      atomicAdd(p.sync.comp_done, mine);
+    }
+  }
+
+  // ---- score: virtual CTAs of FS_WARPS warps, one per CTA while they last
+  NewBlockWait nbw;
+  nbw.ctr = p.sync.comp_done;
+  nbw.target = p.n_groups;
+  nbw.new_seq = p.new_seq;
+  nbw.new_pos = p.new_pos;
+  nbw.n_groups = p.n_groups;
+  const int per_tile = p.W / FS_WARPS;
+  for (int vb = blockIdx.x; vb < p.T * per_tile; vb += gridDim.x) {
+    dec_score_body<FS_WARPS>(a, &tmK, p.ws, p.W, p.chunk, p.nl, vb, smem, nbw);
+    __syncthreads();
+    if (tid < FS_WARPS * DS_NST) {  // the body's mbarriers, before the memory is reused
+      using SM = DecSmemT<FS_WARPS>;
+      uint8_t* al = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~uintptr_t(1023));
+      inval_mbar(al + SM::STAGES + SM::BUF + SM::MLIST + SM::MBOUND + SM::PID + tid * 8);
+    }
+    if (tid == 0) {
+      __threadfence();
+      atomicAdd(&p.sync.tile_done[vb / per_tile], 1);
+    }
+    __syncthreads();
+  }
+
+  // ---- merge: row r by CTA r % gridDim.x, once its tile's lists are all posted
+  for (int row = blockIdx.x; row < a.num_q; row += gridDim.x) {
+    if (tid == 0) wait_geq(&p.sync.tile_done[row / 4], per_tile, a.err);
+    __syncthreads();
+    dec_merge_body(a, p.ws, p.nl, p.lk, row, smem);
+    __syncthreads();
+    if (tid == 0) inval_mbar(smem + MergeSmem::KEYS + MergeSmem::BOUNDS + MergeSmem::HIST + MergeSmem::CAND +
+                             MergeSmem::LISTS + 448);
+    const bool redo = *reinterpret_cast<volatile int32_t*>(&p.ws.redo[row]) != 0;
+    __syncthreads();
+    if (redo) exact_row_body(a, row, p.exact_keys + (long long)row * p.exact_ld, smem);
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      atomicExch(&p.sync.merged[row], 1);
+    }
+  }
+
+  // ---- attend: split i % S of row i / S, once the row is selected
+  const int S = p.aa.splits;
+  for (int it = blockIdx.x; it < a.num_q * S; it += gridDim.x) {
+    const int row = it / S, split = it % S;
+    if (tid == 0) wait_geq(&p.sync.merged[row], 1, a.err);
+    __syncthreads();
+    if (tid < AC::THREADS) sparse_attn_sw_body<D, HKV, SLC>(p.aa, row, split, smem);
+    __syncthreads();
+    if (tid < 2 * AC::NST + 1) inval_mbar(smem + AC::BAR_OFF + tid * 8);
+    __syncthreads();
+  }
+
+  // ---- the last CTA out sets the sync words back to zero for the next launch
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(p.sync.exit_count, 1) == (int)gridDim.x - 1) {
+      *p.sync.comp_done = 0;
+      for (int t = 0; t < p.T; ++t) p.sync.tile_done[t] = 0;
+      for (int r = 0; r < a.num_q; ++r) p.sync.merged[r] = 0;
+      __threadfence();
+      *p.sync.exit_count = 0;
+    }
+  }
+}
+
 }  // namespace
 
 bool score_dec_plan_ok(const Geometry& g) {
@@ -837,6 +1142,154 @@ cudaError_t launch_score_dec(const ScoreArgs& a, const Geometry& g, void* ws, in
   if (e != cudaSuccess) return e;
   dec_merge_kernel<<<g.num_q, DM_THREADS, MergeSmem::TOTAL, s>>>(a, w, p.nl, p.lk);
   return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ fused decode step (host)
+namespace {
+
+struct StepLayout {
+  DecPlan plan;
+  int splits, grid;
+  size_t dec, attn, keys, sync, total;
+  long long exact_ld;
+};
+
+int step_grid() { return num_sms(); }  // one CTA of FS_THREADS per SM
+
+bool step_layout(const Geometry& g, int num_splits, StepLayout* L) {
+  L->grid = step_grid();
+  if (!dec_plan_nw(g, FS_WARPS, (long long)L->grid * FS_WARPS, &L->plan)) return false;
+  L->splits = resolve_sparse_splits(g, num_splits);
+  const DecPlan& p = L->plan;
+  L->dec = stream_region(g) + r256((size_t)p.T * 4 * p.nl * p.lk * 8) + r256((size_t)p.T * 4 * pad2(p.nl) * 8) +
+           r256((size_t)g.num_q * 4);
+  L->attn = r256(sparse_decode_workspace_bytes(g, L->splits));
+  L->exact_ld = (long long)g.max_pos / 4 + 1;
+  L->keys = r256((size_t)g.num_q * L->exact_ld * 8);
+  L->sync = r256((size_t)(2 + p.T + g.num_q) * 4);
+  L->total = L->dec + L->attn + L->keys + L->sync;
+  return true;
+}
+
+template <int D, int HKV>
+cudaError_t launch_step_kernel(const StepArgs& p, const CUtensorMap& tmK, int grid, cudaStream_t s) {
+  constexpr int SLC = kSwSlices<HKV>;
+  using AC = SwCfg<D, HKV, SLC>;
+  int smem = DecSmemT<FS_WARPS>::TOTAL;
+  smem = smem > MergeSmem::TOTAL ? smem : MergeSmem::TOTAL;
+  smem = smem > ExactSmem::TOTAL ? smem : ExactSmem::TOTAL;
+  smem = smem > AC::TOTAL ? smem : AC::TOTAL;
+  cudaError_t e = set_smem_once(decode_step_kernel<D, HKV, SLC>, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(FS_THREADS);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the waits between them end
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_step_kernel<D, HKV, SLC>, p, tmK);
+}
+
+}  // namespace
+
+bool decode_step_supported(const Geometry& g) {
+  StepLayout L;
+  return g.Di == 128 && g.G <= 8 && g.topk <= 512 && g.num_q <= 256 && step_layout(g, 0, &L);
+}
+
+size_t decode_step_workspace_bytes(const Geometry& g, int num_splits) {
+  StepLayout L;
+  if (!step_layout(g, num_splits, &L)) return 0;
+  return L.total;
+}
+
+cudaError_t launch_decode_step(const Geometry& g, const void* idx_k_new, const int32_t* new_seq,
+                               const int32_t* new_pos, int n_new, void* kcomp, const void* idx_q,
+                               const void* idx_w, const void* q, const void* k_pool,
+                               const void* v_pool, int32_t* sel, int32_t* n_sel, float* sel_scores,
+                               void* out, float* lse, int num_splits, void* ws, cudaStream_t s) {
+  auto enc = tmap_encode_fn();
+  StepLayout L;
+  if (!enc || !step_layout(g, num_splits, &L)) return cudaErrorNotSupported;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  StepArgs p;
+  p.sa = make_args(g, idx_q, idx_w, kcomp, sel, n_sel, sel_scores);
+  p.ws = carve_dec(g, L.plan, base);
+  p.W = L.plan.W;
+  p.chunk = L.plan.chunk;
+  p.nl = L.plan.nl;
+  p.lk = L.plan.lk;
+  p.T = L.plan.T;
+  p.idx_k_new = static_cast<const bf16*>(idx_k_new);
+  p.new_seq = new_seq;
+  p.new_pos = new_pos;
+  p.n_groups = n_new / 4;
+  p.kcomp_w = static_cast<bf16*>(kcomp);
+  p.exact_keys = reinterpret_cast<u64*>(base + L.dec + L.attn);
+  p.exact_ld = L.exact_ld;
+  int* sync = reinterpret_cast<int*>(base + L.dec + L.attn + L.keys);
+  p.sync.comp_done = sync;
+  p.sync.exit_count = sync + 1;
+  p.sync.tile_done = sync + 2;
+  p.sync.merged = sync + 2 + L.plan.T;
+  AttnArgs& aa = p.aa;
+  aa.q = static_cast<const bf16*>(q);
+  aa.k_pool = static_cast<const bf16*>(k_pool);
+  aa.v_pool = static_cast<const bf16*>(v_pool);
+  aa.sel = sel;
+  aa.n_sel = n_sel;
+  aa.sel_stride = g.topk + 1;
+  aa.q_seq = g.q_seq;
+  aa.q_pos = g.q_pos;
+  aa.page_table = g.page_table;
+  aa.num_q = g.num_q;
+  aa.batch = g.batch;
+  aa.max_pages = g.max_pages;
+  aa.num_pages = g.num_pages;
+  aa.Hq = g.Hq;
+  aa.G = g.G;
+  aa.scale_log2 = g.scale_log2;
+  aa.out = static_cast<bf16*>(out);
+  aa.lse = lse;
+  aa.splits = L.splits;
+  aa.err = g.err;
+  aa.part_o = nullptr;
+  aa.part_lse = nullptr;
+  aa.arrivals = nullptr;
+  if (L.splits > 1) {
+    const size_t n = (size_t)g.num_q * L.splits * g.Hq;
+    uint8_t* ab = base + L.dec;
+    aa.part_o = reinterpret_cast<float*>(ab);
+    aa.part_lse = reinterpret_cast<float*>(ab + ((n * g.D * 4 + 255) / 256) * 256);
+    aa.arrivals = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(aa.part_lse) + ((n * 4 + 255) / 256) * 256);
+  }
+  CUtensorMap tmK;
+  {
+    cuuint64_t dims[2] = {128, (cuuint64_t)g.num_pages * 16};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, 16};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kcomp, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+#define QSA_STEP_CASE(DD, HH) \
+  if (g.D == DD && g.Hkv == HH) return launch_step_kernel<DD, HH>(p, tmK, L.grid, s);
+  QSA_STEP_CASE(128, 4)
+  QSA_STEP_CASE(128, 8)
+  QSA_STEP_CASE(128, 2)
+  QSA_STEP_CASE(128, 1)
+  QSA_STEP_CASE(64, 4)
+  QSA_STEP_CASE(64, 8)
+  QSA_STEP_CASE(64, 2)
+  QSA_STEP_CASE(64, 1)
+#undef QSA_STEP_CASE
+  return cudaErrorNotSupported;
 }
 
 }  // namespace qsa
