@@ -311,6 +311,62 @@ def graph_decode_us(w: Workload, steps: int, warmup: int, flush):
     return statistics.mean(us), us
 
 
+def fused_decode_us(w: Workload, steps: int, warmup: int, flush):
+    """The fused one-launch decode step (qsa_decode_step), replayed as a one-node CUDA graph with
+    L2 flushed before each replay (eager launches when the graph cannot be captured).  Checks its
+    output against the three-call step's before timing."""
+    torch = w.torch
+    from learned_block_sparse_qsa_b200 import QSA_OP_DECODE_STEP, qsa_decode_step, qsa_workspace_size
+
+    c, d, b = w.c, w.di, w.b
+    n = qsa_workspace_size(w.cfg, b, QSA_OP_DECODE_STEP, 0)
+    ws = torch.zeros(n, dtype=torch.uint8, device=d.q.device)
+    out = torch.empty_like(w.out)
+
+    def one():
+        qsa_decode_step(w.cfg, b, d.idx_k_new, d.new_seq, d.new_pos, d.new_seq.numel(), d.kcomp_pool,
+                        d.idx_q, d.idx_w, d.q, d.k_pool, d.v_pool, w.sel, w.n_sel, None, out, None, 0,
+                        ws, n)
+
+    one()
+    w.step(True)
+    torch.cuda.synchronize()
+    if not torch.equal(out.view(torch.int16), w.out.view(torch.int16)):
+        raise RuntimeError("fused decode step output differs from the three-call step")
+    mode = "cuda_graph"
+    g = None
+    try:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            one()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            one()
+    except Exception as e:  # pragma: no cover - capture support depends on the driver
+        log(f"fused step not capturable ({e}); timing eager launches")
+        g, mode = None, "eager"
+        torch.cuda.synchronize()
+    run = g.replay if g is not None else one
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        a.record()
+        run()
+        e.record()
+        ts.append((a, e))
+    torch.cuda.synchronize()
+    del g
+    return statistics.mean(x.elapsed_time(y) * 1000 for x, y in ts), mode
+
+
 class Staging:
     """One pinned host buffer holding every per-step input of a workload, and device buffers it is
     copied into with a single host-to-device copy; tensors are 256-byte aligned views."""
@@ -762,6 +818,8 @@ def main():
     log("decode eager stages " + ", ".join(f"{k} {v * 1000:.1f} us" for k, v in dstage_ms.items()))
     graph_us, _ = graph_decode_us(wd, dsteps, args.warmup, flush)
     log(f"decode graph {graph_us:.1f} us/step")
+    fused_us, fused_mode = fused_decode_us(wd, dsteps, args.warmup, flush)
+    log(f"decode fused step {fused_us:.1f} us/step ({fused_mode})")
     graph_us = max_over_ranks(graph_us, dist)
     d_e2e_us, dh2d, dd2h = e2e_decode(wd, dsteps, args.warmup)
     d_e2e_us = max_over_ranks(d_e2e_us, dist)
@@ -821,6 +879,7 @@ def main():
                                "dense_decode_gbs": workd["dense_bytes_decode"] / (dense_dec_ms * 1e-3) / 1e9,
                                "article_ratios_context": {"prefill": 7.6, "decode": 4.9}},
             "decode": {"workload": cd.name, "us_per_step": graph_us, "cuda_graph": True,
+                       "fused_step_us": fused_us, "fused_step_timing": fused_mode,
                        "us_per_step_eager": statistics.mean(dstep_ms) * 1000,
                        "stages_us": {k: v["ms"] * 1000 for k, v in dstages.items()},
                        "stages": dstages, "path_roofline_us": dpath_roof_us,

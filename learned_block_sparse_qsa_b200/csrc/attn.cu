@@ -432,6 +432,8 @@ cudaError_t launch_sparse_attn(const Geometry& g, const void* q, const void* k_p
   a.part_o = nullptr;
   a.part_lse = nullptr;
   a.arrivals = nullptr;
+  a.coop = 0;
+  a.departures = nullptr;
   if (splits > 1) {
     const size_t n = (size_t)g.num_q * splits * g.Hq;
     a.part_o = static_cast<float*>(ws);

@@ -25,6 +25,12 @@ struct AttnArgs {
   float* part_lse;
   int splits;
   uint32_t* arrivals;  // split-K: per-row count of finished splits (zeroed before the launch)
+  // Cooperative combine (only when every split of a row is resident at once, as in a cooperative
+  // launch with one split per CTA): each split waits for all of its row's partials, then merges
+  // the heads h = split (mod splits); `departures` counts the splits done reading, and the last
+  // one sets both counters back to zero.  0 / nullptr: the last split merges every head.
+  int coop;
+  uint32_t* departures;
   int32_t* err;
 };
 
@@ -364,7 +370,60 @@ __device__ __forceinline__ void sparse_attn_sw_body(const AttnArgs& a, const int
   }
   }  // consumers
 
-  if (a.splits > 1) {
+  if (a.splits > 1 && a.coop) {
+    __threadfence();
+    sw_cta_sync<C::THREADS>();
+    if (tid == 0) {
+      atomicAdd(&a.arrivals[row], 1u);
+      const volatile uint32_t* ar = a.arrivals + row;
+      const long long t0 = clock64();
+      while (*ar < (uint32_t)a.splits) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+          flag_error(a.err, QSA_DEVERR_TIMEOUT);
+          break;
+        }
+      }
+      __threadfence();
+    }
+    sw_cta_sync<C::THREADS>();
+    const int S = a.splits, Hq = a.Hq;
+    const long long b0 = (long long)row * S * Hq;  // partial index of (split 0, head 0)
+    const int nh = (Hq - split + S - 1) / S;       // this split's heads: split, split + S, ...
+    constexpr int D4 = D / 4;
+    for (int e = tid; e < nh * D4; e += C::THREADS) {
+      const int hq = split + (e / D4) * S, d = (e % D4) * 4;
+      float M = -INFINITY;
+      for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(a.part_lse + b0 + (long long)sp * Hq + hq));
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (M != -INFINITY) {
+        for (int sp = 0; sp < S; ++sp) {
+          const long long pi = b0 + (long long)sp * Hq + hq;
+          const float v = __ldcg(a.part_lse + pi);
+          if (v == -INFINITY) continue;
+          const float w = exp2f(v - M);
+          L += w;
+          const float4 o = __ldcg(reinterpret_cast<const float4*>(a.part_o + pi * D + d));
+          acc.x = fmaf(w, o.x, acc.x);
+          acc.y = fmaf(w, o.y, acc.y);
+          acc.z = fmaf(w, o.z, acc.z);
+          acc.w = fmaf(w, o.w, acc.w);
+        }
+      }
+      const float inv = L > 0.f ? 1.0f / L : 0.f;
+      uint2 packed;
+      packed.x = pack_bf16(acc.x * inv, acc.y * inv);
+      packed.y = pack_bf16(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(a.out + ((long long)row * Hq + hq) * D + d) = packed;
+      if (d == 0 && a.lse)
+        a.lse[(long long)row * Hq + hq] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    }
+    sw_cta_sync<C::THREADS>();
+    if (tid == 0 && atomicAdd(&a.departures[row], 1u) == (uint32_t)S - 1u) {
+      a.arrivals[row] = 0u;  // every split of the row has read its partials
+      a.departures[row] = 0u;
+    }
+  } else if (a.splits > 1) {
     // the last split of the row to finish merges all of the row's partials (log-sum-exp weights)
     __shared__ int s_last;
     __threadfence();

@@ -191,13 +191,16 @@ struct NewBlockWait {
 
 // The streaming part of the decode indexer for virtual CTA `vblock` of NW warps (all threads of
 // the calling block take part).  smem_raw: DecSmemT<NW>::TOTAL bytes.
+// ltid: the thread's index within the NW warps running the body (warp-aligned); bar_id: the named
+// barrier over those NW * 32 threads (0: the whole block is exactly those threads).
 template <int NW>
 __device__ __forceinline__ void dec_score_body(const ScoreArgs& a, const CUtensorMap* tmK, const DecWs& ws,
                                                int W, int chunk, int nl, int vblock, uint8_t* smem_raw,
-                                               const NewBlockWait& nbw) {
+                                               const NewBlockWait& nbw, const int ltid = threadIdx.x,
+                                               const int bar_id = 0) {
   using DecSmem = DecSmemT<NW>;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = ltid >> 5, lane = ltid & 31;
   const int gw = vblock * NW + warp;
   const int T = (a.num_q + 3) / 4;
   const int tile = gw / W, wc = gw % W;
@@ -446,7 +449,8 @@ __device__ __forceinline__ void dec_score_body(const ScoreArgs& a, const CUtenso
 
   if (!cta_merge) return;
   // CTA merge: warp r (< 4) folds the NW lists of row r into one list of DS_KC keys
-  __syncthreads();
+  if (bar_id == 0) __syncthreads();
+  else asm volatile("bar.sync %0, %1;\n" ::"r"(bar_id), "n"(NW * 32) : "memory");
   const int r = warp;
   if (r >= 4 || tile * 4 + r >= a.num_q) return;
   u64 top = 0, bound = 0;
@@ -1035,18 +1039,25 @@ __global__ void __launch_bounds__(FS_THREADS, 1)
   nbw.new_seq = p.new_seq;
   nbw.new_pos = p.new_pos;
   nbw.n_groups = p.n_groups;
-  const int per_tile = p.W / FS_WARPS;
-  for (int vb = blockIdx.x; vb < p.T * per_tile; vb += gridDim.x) {
-    dec_score_body<FS_WARPS>(a, &tmK, p.ws, p.W, p.chunk, p.nl, vb, smem, nbw);
-    __syncthreads();
-    if (tid < FS_WARPS * DS_NST) {  // the body's mbarriers, before the memory is reused
-      using SM = DecSmemT<FS_WARPS>;
-      uint8_t* al = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~uintptr_t(1023));
-      inval_mbar(al + SM::STAGES + SM::BUF + SM::MLIST + SM::MBOUND + SM::PID + tid * 8);
-    }
-    if (tid == 0) {
-      __threadfence();
-      atomicAdd(&p.sync.tile_done[vb / per_tile], 1);
+  // two virtual CTAs of DS_WARPS warps per block, as the standalone kernel runs two CTAs per SM:
+  // a half that finishes its chunk folds its lists while the other half still streams
+  const int per_tile = p.W / DS_WARPS;
+  const int half = tid / DS_THREADS, htid = tid % DS_THREADS;
+  uint8_t* hsmem = smem + half * DecSmem::TOTAL;
+  for (int vb0 = 2 * blockIdx.x; vb0 < p.T * per_tile; vb0 += 2 * gridDim.x) {
+    const int vb = vb0 + half;
+    if (vb < p.T * per_tile) {
+      dec_score_body<DS_WARPS>(a, &tmK, p.ws, p.W, p.chunk, p.nl, vb, hsmem, nbw, htid, 1 + half);
+      asm volatile("bar.sync %0, %1;\n" ::"r"(1 + half), "n"(DS_THREADS) : "memory");
+      if (htid < DS_WARPS * DS_NST) {  // the body's mbarriers, before the memory is reused
+        uint8_t* al = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(hsmem) + 1023) & ~uintptr_t(1023));
+        inval_mbar(al + DecSmem::STAGES + DecSmem::BUF + DecSmem::MLIST + DecSmem::MBOUND + DecSmem::PID +
+                   htid * 8);
+      }
+      if (htid == 0) {
+        __threadfence();
+        atomicAdd(&p.sync.tile_done[vb / per_tile], 1);
+      }
     }
     __syncthreads();
   }
@@ -1158,7 +1169,7 @@ int step_grid() { return num_sms(); }  // one CTA of FS_THREADS per SM
 
 bool step_layout(const Geometry& g, int num_splits, StepLayout* L) {
   L->grid = step_grid();
-  if (!dec_plan_nw(g, FS_WARPS, (long long)L->grid * FS_WARPS, &L->plan)) return false;
+  if (!dec_plan_nw(g, DS_WARPS, (long long)L->grid * FS_WARPS, &L->plan)) return false;
   L->splits = resolve_sparse_splits(g, num_splits);
   const DecPlan& p = L->plan;
   L->dec = stream_region(g) + r256((size_t)p.T * 4 * p.nl * p.lk * 8) + r256((size_t)p.T * 4 * pad2(p.nl) * 8) +
@@ -1166,7 +1177,7 @@ bool step_layout(const Geometry& g, int num_splits, StepLayout* L) {
   L->attn = r256(sparse_decode_workspace_bytes(g, L->splits));
   L->exact_ld = (long long)g.max_pos / 4 + 1;
   L->keys = r256((size_t)g.num_q * L->exact_ld * 8);
-  L->sync = r256((size_t)(2 + p.T + g.num_q) * 4);
+  L->sync = r256((size_t)(2 + p.T + 2 * g.num_q) * 4);
   L->total = L->dec + L->attn + L->keys + L->sync;
   return true;
 }
@@ -1175,7 +1186,7 @@ template <int D, int HKV>
 cudaError_t launch_step_kernel(const StepArgs& p, const CUtensorMap& tmK, int grid, cudaStream_t s) {
   constexpr int SLC = kSwSlices<HKV>;
   using AC = SwCfg<D, HKV, SLC>;
-  int smem = DecSmemT<FS_WARPS>::TOTAL;
+  int smem = 2 * DecSmem::TOTAL;
   smem = smem > MergeSmem::TOTAL ? smem : MergeSmem::TOTAL;
   smem = smem > ExactSmem::TOTAL ? smem : ExactSmem::TOTAL;
   smem = smem > AC::TOTAL ? smem : AC::TOTAL;
@@ -1236,6 +1247,7 @@ cudaError_t launch_decode_step(const Geometry& g, const void* idx_k_new, const i
   p.sync.exit_count = sync + 1;
   p.sync.tile_done = sync + 2;
   p.sync.merged = sync + 2 + L.plan.T;
+  uint32_t* departures = reinterpret_cast<uint32_t*>(sync + 2 + L.plan.T + g.num_q);
   AttnArgs& aa = p.aa;
   aa.q = static_cast<const bf16*>(q);
   aa.k_pool = static_cast<const bf16*>(k_pool);
@@ -1260,6 +1272,8 @@ cudaError_t launch_decode_step(const Geometry& g, const void* idx_k_new, const i
   aa.part_o = nullptr;
   aa.part_lse = nullptr;
   aa.arrivals = nullptr;
+  aa.coop = (long long)g.num_q * L.splits <= L.grid;  // one split per CTA: all resident at once
+  aa.departures = departures;
   if (L.splits > 1) {
     const size_t n = (size_t)g.num_q * L.splits * g.Hq;
     uint8_t* ab = base + L.dec;
