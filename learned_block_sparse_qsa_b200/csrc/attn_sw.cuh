@@ -392,28 +392,29 @@ __device__ __forceinline__ void sparse_attn_sw_body(const AttnArgs& a, const int
     constexpr int D4 = D / 4;
     for (int e = tid; e < nh * D4; e += C::THREADS) {
       const int hq = split + (e / D4) * S, d = (e % D4) * 4;
+      // the same weights, in the same order, as the last-split merge below: bit-identical output
       float M = -INFINITY;
       for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(a.part_lse + b0 + (long long)sp * Hq + hq));
       float L = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (M != -INFINITY) {
-        for (int sp = 0; sp < S; ++sp) {
-          const long long pi = b0 + (long long)sp * Hq + hq;
-          const float v = __ldcg(a.part_lse + pi);
-          if (v == -INFINITY) continue;
-          const float w = exp2f(v - M);
-          L += w;
-          const float4 o = __ldcg(reinterpret_cast<const float4*>(a.part_o + pi * D + d));
-          acc.x = fmaf(w, o.x, acc.x);
-          acc.y = fmaf(w, o.y, acc.y);
-          acc.z = fmaf(w, o.z, acc.z);
-          acc.w = fmaf(w, o.w, acc.w);
-        }
+      for (int sp = 0; sp < S; ++sp) {
+        const float v = __ldcg(a.part_lse + b0 + (long long)sp * Hq + hq);
+        L += (M != -INFINITY && v != -INFINITY) ? exp2f(v - M) : 0.f;
       }
       const float inv = L > 0.f ? 1.0f / L : 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < S; ++sp) {
+        const long long pi = b0 + (long long)sp * Hq + hq;
+        const float v = __ldcg(a.part_lse + pi);
+        const float w = ((M != -INFINITY && v != -INFINITY) ? exp2f(v - M) : 0.f) * inv;
+        const float4 o = __ldcg(reinterpret_cast<const float4*>(a.part_o + pi * D + d));
+        acc.x = fmaf(w, o.x, acc.x);
+        acc.y = fmaf(w, o.y, acc.y);
+        acc.z = fmaf(w, o.z, acc.z);
+        acc.w = fmaf(w, o.w, acc.w);
+      }
       uint2 packed;
-      packed.x = pack_bf16(acc.x * inv, acc.y * inv);
-      packed.y = pack_bf16(acc.z * inv, acc.w * inv);
+      packed.x = pack_bf16(acc.x, acc.y);
+      packed.y = pack_bf16(acc.z, acc.w);
       *reinterpret_cast<uint2*>(a.out + ((long long)row * Hq + hq) * D + d) = packed;
       if (d == 0 && a.lse)
         a.lse[(long long)row * Hq + hq] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
