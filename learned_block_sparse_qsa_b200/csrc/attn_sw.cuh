@@ -390,34 +390,71 @@ __device__ __forceinline__ void sparse_attn_sw_body(const AttnArgs& a, const int
     const long long b0 = (long long)row * S * Hq;  // partial index of (split 0, head 0)
     const int nh = (Hq - split + S - 1) / S;       // this split's heads: split, split + S, ...
     constexpr int D4 = D / 4;
-    for (int e = tid; e < nh * D4; e += C::THREADS) {
-      const int hq = split + (e / D4) * S, d = (e % D4) * 4;
-      // the same weights, in the same order, as the last-split merge below: bit-identical output
-      float M = -INFINITY;
-      for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(a.part_lse + b0 + (long long)sp * Hq + hq));
-      float L = 0.f;
+    const long long step = (long long)Hq * D / 4;  // float4s between splits
+    // the first PRE partials of this thread's first output group are loaded before anything else,
+    // so that their latency overlaps the weights' computation
+    constexpr int PRE = 8;
+    float4 pre[PRE];
+    {
+      const int e = tid;
+      if (e < nh * D4) {
+        const float4* src = reinterpret_cast<const float4*>(a.part_o + (b0 + split + (e / D4) * S) * D + (e % D4) * 4);
+#pragma unroll
+        for (int j = 0; j < PRE; ++j) pre[j] = j < S ? __ldcg(src + j * step) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    // the heads' S log-sum-exps, loaded at once into the idle stage ring, then turned into the
+    // last-split merge's weights (same values, same order: the output is bit-identical)
+    float* wn = reinterpret_cast<float*>(smem);    // [nh][S]
+    for (int i = tid; i < nh * S; i += C::THREADS) {
+      const int hi = i / S, sp = i % S;
+      wn[i] = __ldcg(a.part_lse + b0 + (long long)sp * Hq + split + hi * S);
+    }
+    sw_cta_sync<C::THREADS>();
+    if (tid < nh) {
+      float* w = wn + tid * S;
+      float M = -INFINITY, L = 0.f;
+      for (int sp = 0; sp < S; ++sp) M = fmaxf(M, w[sp]);
       for (int sp = 0; sp < S; ++sp) {
-        const float v = __ldcg(a.part_lse + b0 + (long long)sp * Hq + hq);
-        L += (M != -INFINITY && v != -INFINITY) ? exp2f(v - M) : 0.f;
+        const float e = (M != -INFINITY && w[sp] != -INFINITY) ? exp2f(w[sp] - M) : 0.f;
+        w[sp] = e;
+        L += e;
       }
       const float inv = L > 0.f ? 1.0f / L : 0.f;
+      for (int sp = 0; sp < S; ++sp) w[sp] *= inv;
+      if (a.lse)
+        a.lse[(long long)row * Hq + split + tid * S] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    }
+    sw_cta_sync<C::THREADS>();
+    for (int e = tid; e < nh * D4; e += C::THREADS) {
+      const int hi = e / D4, hq = split + hi * S, d = (e % D4) * 4;
+      const float* w = wn + hi * S;
+      const float4* src = reinterpret_cast<const float4*>(a.part_o + (b0 + hq) * D + d);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp = 0; sp < S; ++sp) {
-        const long long pi = b0 + (long long)sp * Hq + hq;
-        const float v = __ldcg(a.part_lse + pi);
-        const float w = ((M != -INFINITY && v != -INFINITY) ? exp2f(v - M) : 0.f) * inv;
-        const float4 o = __ldcg(reinterpret_cast<const float4*>(a.part_o + pi * D + d));
-        acc.x = fmaf(w, o.x, acc.x);
-        acc.y = fmaf(w, o.y, acc.y);
-        acc.z = fmaf(w, o.z, acc.z);
-        acc.w = fmaf(w, o.w, acc.w);
+      int sp = 0;
+      if (e == tid) {  // the preloaded group
+#pragma unroll
+        for (int j = 0; j < PRE; ++j) {
+          if (j < S) {
+            acc.x = fmaf(w[j], pre[j].x, acc.x);
+            acc.y = fmaf(w[j], pre[j].y, acc.y);
+            acc.z = fmaf(w[j], pre[j].z, acc.z);
+            acc.w = fmaf(w[j], pre[j].w, acc.w);
+          }
+        }
+        sp = S < PRE ? S : PRE;
+      }
+      for (; sp < S; ++sp) {
+        const float4 p = __ldcg(src + sp * step);
+        acc.x = fmaf(w[sp], p.x, acc.x);
+        acc.y = fmaf(w[sp], p.y, acc.y);
+        acc.z = fmaf(w[sp], p.z, acc.z);
+        acc.w = fmaf(w[sp], p.w, acc.w);
       }
       uint2 packed;
       packed.x = pack_bf16(acc.x, acc.y);
       packed.y = pack_bf16(acc.z, acc.w);
       *reinterpret_cast<uint2*>(a.out + ((long long)row * Hq + hq) * D + d) = packed;
-      if (d == 0 && a.lse)
-        a.lse[(long long)row * Hq + hq] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
     sw_cta_sync<C::THREADS>();
     if (tid == 0 && atomicAdd(&a.departures[row], 1u) == (uint32_t)S - 1u) {

@@ -478,7 +478,9 @@ __global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
 
 // ------------------------------------------------------------------ merge (one CTA per row)
 
-constexpr int DM_CAND = 512;  // keys of the boundary histogram bin ranked directly
+constexpr int DM_CAND = 512;        // capacity of the boundary-bin key list
+constexpr int DM_RANK_DIRECT = 64;  // a boundary bin this small is ranked by direct comparison;
+                                    // a larger one costs O(n^2) there and is refined instead
 
 struct MergeSmem {
   static constexpr int KEYS = DM_MAXU * 8;
@@ -545,37 +547,21 @@ __device__ __forceinline__ u64 cta_max_u64(u64 v, u64* red) {
   return m;
 }
 
-// The need-th largest of n unique keys in shared memory (1 <= need <= n), by the whole CTA:
-// MSB-first radix select with 11-bit digits starting at the highest bit where the keys differ.
-__device__ u64 cta_kth_largest(const u64* keys, int n, int need, uint32_t* hist, u64* red,
-                               uint32_t* wsum, uint32_t* sel3) {
+// Radix-select continuation: among the keys k with (k & mask) == prefix -- the bits above bit
+// `top` already decided -- the `remaining`-th largest, by 11-bit digits from bit `top` down.
+__device__ u64 cta_kth_refine(const u64* keys, int n, uint32_t remaining, u64 prefix, u64 mask, int top,
+                              uint32_t* hist, u64* red, uint32_t* wsum, uint32_t* sel3) {
   const int tid = threadIdx.x;
-  u64 lo = ~0ull, hi = 0ull;
-  for (int i = tid; i < n; i += DM_THREADS) {
-    const u64 k = keys[i];
-    lo = k < lo ? k : lo;
-    hi = k > hi ? k : hi;
-  }
-  lo = cta_min_u64(lo, red);
-  hi = cta_max_u64(hi, red);
-  if (need == n) return lo;
-  if (need == 1) return hi;
-  int top = 63 - __clzll((long long)(lo ^ hi));
-  u64 prefix = 0, mask = 0;
-  if (top < 63) {
-    mask = ~((2ull << top) - 1ull);
-    prefix = hi & mask;
-  }
-  uint32_t remaining = (uint32_t)need;
   for (;;) {
     const int width = top + 1 < 11 ? top + 1 : 11;
     const int shift = top + 1 - width;
     const int nb = 1 << width;
     for (int i = tid; i < nb; i += DM_THREADS) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += DM_THREADS) {
-      const u64 k = keys[i];
-      if ((k & mask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & (uint32_t)(nb - 1)], 1u);
+    for (int base = 0; base < n; base += DM_THREADS) {
+      const int i = base + tid;
+      const u64 k = i < n ? keys[i] : 0ull;
+      hist_add(hist, (uint32_t)(k >> shift) & (uint32_t)(nb - 1), i < n && (k & mask) == prefix);
     }
     __syncthreads();
     const int per = (nb + DM_THREADS - 1) / DM_THREADS;  // bins per thread, counted from the top
@@ -616,6 +602,30 @@ __device__ u64 cta_kth_largest(const u64* keys, int n, int need, uint32_t* hist,
     }
     top = shift - 1;
   }
+}
+
+// The need-th largest of n unique keys in shared memory (1 <= need <= n), by the whole CTA:
+// MSB-first radix select with 11-bit digits starting at the highest bit where the keys differ.
+__device__ u64 cta_kth_largest(const u64* keys, int n, int need, uint32_t* hist, u64* red,
+                               uint32_t* wsum, uint32_t* sel3) {
+  const int tid = threadIdx.x;
+  u64 lo = ~0ull, hi = 0ull;
+  for (int i = tid; i < n; i += DM_THREADS) {
+    const u64 k = keys[i];
+    lo = k < lo ? k : lo;
+    hi = k > hi ? k : hi;
+  }
+  lo = cta_min_u64(lo, red);
+  hi = cta_max_u64(hi, red);
+  if (need == n) return lo;
+  if (need == 1) return hi;
+  const int top = 63 - __clzll((long long)(lo ^ hi));
+  u64 prefix = 0, mask = 0;
+  if (top < 63) {
+    mask = ~((2ull << top) - 1ull);
+    prefix = hi & mask;
+  }
+  return cta_kth_refine(keys, n, (uint32_t)need, prefix, mask, top, hist, red, wsum, sel3);
 }
 
 // One CTA per query row.  The row's lists come in block order (list l covers a block range below
@@ -751,9 +761,10 @@ __device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& 
     const u64 prefix = hi & hmask;
     for (uint32_t i = tid; i < nb; i += DM_THREADS) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < U; i += DM_THREADS) {
-      const u64 k = keys[i];
-      if (k && (k & hmask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & (nb - 1)], 1u);
+    for (int base = 0; base < U; base += DM_THREADS) {
+      const int i = base + tid;
+      const u64 k = i < U ? keys[i] : 0ull;
+      hist_add(hist, (uint32_t)(k >> shift) & (nb - 1), i < U && k && (k & hmask) == prefix);
     }
     __syncthreads();
     const int per = (int)(nb + DM_THREADS - 1) / DM_THREADS;  // bins per thread from the top
@@ -780,7 +791,7 @@ __device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& 
     if (tid == 0) sel3[3] = 0;
     __syncthreads();
     const uint32_t digit = sel3[0], above = sel3[1], inbin = sel3[2];
-    if (inbin <= (uint32_t)DM_THREADS) {
+    if (inbin <= (uint32_t)DM_RANK_DIRECT) {
       // the boundary bin's keys, each ranked by counting the larger ones (keys are unique)
       const u64 bmask = hmask | ((u64)(nb - 1) << shift);
       const u64 bpre = prefix | ((u64)digit << shift);
@@ -797,8 +808,13 @@ __device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& 
       }
       __syncthreads();
       tau = *s_tau;
-    } else {  // a crowded bin: the full CTA radix select
-      tau = cta_kth_largest(keys, U, need, hist, red, wsum, sel3);
+    } else {  // a crowded bin: refine by the next digits below it
+      __syncthreads();
+      const u64 bmask = hmask | ((u64)(nb - 1) << shift);
+      const u64 bpre = prefix | ((u64)digit << shift);
+      tau = shift == 0 ? bpre
+                       : cta_kth_refine(keys, U, (uint32_t)need - above, bpre, bmask, shift - 1, hist, red,
+                                        wsum, sel3);
     }
   }
   if (mb > tau) {  // a dropped key could beat tau: the exact kernel redoes the row
