@@ -558,10 +558,9 @@ __device__ u64 cta_kth_refine(const u64* keys, int n, uint32_t remaining, u64 pr
     const int nb = 1 << width;
     for (int i = tid; i < nb; i += DM_THREADS) hist[i] = 0;
     __syncthreads();
-    for (int base = 0; base < n; base += DM_THREADS) {
-      const int i = base + tid;
-      const u64 k = i < n ? keys[i] : 0ull;
-      hist_add(hist, (uint32_t)(k >> shift) & (uint32_t)(nb - 1), i < n && (k & mask) == prefix);
+    for (int i = tid; i < n; i += DM_THREADS) {
+      const u64 k = keys[i];
+      if ((k & mask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & (uint32_t)(nb - 1)], 1u);
     }
     __syncthreads();
     const int per = (nb + DM_THREADS - 1) / DM_THREADS;  // bins per thread, counted from the top
@@ -761,10 +760,9 @@ __device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& 
     const u64 prefix = hi & hmask;
     for (uint32_t i = tid; i < nb; i += DM_THREADS) hist[i] = 0;
     __syncthreads();
-    for (int base = 0; base < U; base += DM_THREADS) {
-      const int i = base + tid;
-      const u64 k = i < U ? keys[i] : 0ull;
-      hist_add(hist, (uint32_t)(k >> shift) & (nb - 1), i < U && k && (k & hmask) == prefix);
+    for (int i = tid; i < U; i += DM_THREADS) {
+      const u64 k = keys[i];
+      if (k && (k & hmask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & (nb - 1)], 1u);
     }
     __syncthreads();
     const int per = (int)(nb + DM_THREADS - 1) / DM_THREADS;  // bins per thread from the top

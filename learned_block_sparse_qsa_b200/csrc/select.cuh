@@ -10,14 +10,9 @@ namespace qsa {
 
 typedef unsigned long long u64;
 
-// Histogram increment (shared-memory atomic).  Called by all 32 lanes of the warp; lanes that hit
-// the same bin are combined into one atomic, since the keys near a row's threshold crowd into a
-// few bins and same-address atomics serialise.
+// Histogram increment (shared-memory atomic).  Called by all 32 lanes of the warp.
 __device__ __forceinline__ void hist_add(uint32_t* h, uint32_t bin, bool active) {
-  const unsigned act = __ballot_sync(0xffffffffu, active);
-  if (!active) return;
-  const unsigned peers = __match_any_sync(act, bin);
-  if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], (uint32_t)__popc(peers));
+  if (active) atomicAdd(&h[bin], 1u);
 }
 
 // One warp: find the `need`-th largest of the `cnt` unique keys in buf[0..cnt) by an MSB-first
@@ -161,10 +156,9 @@ __device__ __forceinline__ u64 warp_kth_largest2(const u64* ka, int na, const u6
     const uint32_t nb = 1u << width;
     for (uint32_t i = lane; i < nb; i += 32) hist[i] = 0;
     __syncwarp();
-    for (int base = 0; base < n; base += 32) {
-      const int i = base + lane;
-      const u64 k = i < n ? key_at(i) : 0ull;
-      hist_add(hist, (uint32_t)(k >> shift) & (nb - 1), i < n && (k & mask) == prefix);
+    for (int i = lane; i < n; i += 32) {
+      const u64 k = key_at(i);
+      if ((k & mask) == prefix) atomicAdd(&hist[(uint32_t)(k >> shift) & (nb - 1)], 1u);
     }
     __syncwarp();
     // lane l owns a contiguous run of bins counted from the top
