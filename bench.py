@@ -696,6 +696,27 @@ def training_kernels(w: Workload, peaks, reps: int = 3):
     }
 
 
+def training_kernels_case(w: Workload, reps: int):
+    """The attention backward and the distillation signal on one --case workload (ncu target)."""
+    torch = w.torch
+    from learned_block_sparse_qsa_b200 import (qsa_index_distill_kl, qsa_sparse_attn_backward,
+                                               qsa_sparse_attn_prefill)
+
+    c, d, b = w.c, w.di, w.b
+    lse = torch.empty(c.num_q, c.Hq, dtype=torch.float32, device=d.q.device)
+    qsa_sparse_attn_prefill(w.cfg, b, d.q, d.k_pool, d.v_pool, w.sel, w.n_sel, w.out, lse)
+    dout = torch.ones(d.q.shape, dtype=torch.bfloat16, device=d.q.device)
+    dq = torch.empty(d.q.shape, dtype=torch.float32, device=d.q.device)
+    dk = torch.zeros(d.k_pool.shape, dtype=torch.float32, device=d.q.device)
+    dv = torch.zeros_like(dk)
+    kl = torch.empty(c.num_q, dtype=torch.float32, device=d.q.device)
+    bwd = _time_ms(torch, lambda: qsa_sparse_attn_backward(w.cfg, b, d.q, d.k_pool, d.v_pool, w.sel, w.n_sel,
+                                                           w.out, lse, dout, dq, dk, dv), reps)
+    dst = _time_ms(torch, lambda: qsa_index_distill_kl(w.cfg, b, d.q, d.k_pool, d.idx_q, d.idx_w,
+                                                       d.kcomp_pool, kl), reps)
+    return {"sparse_attn_backward_ms": bwd, "distill_kl_ms": dst}
+
+
 # ------------------------------------------------------------------------------------ main
 
 def main():
@@ -706,6 +727,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--case", default="", help="time one workload (C1..C5) only, per stage")
     ap.add_argument("--chunk", type=int, default=0, help="with --case: new tokens per sequence")
+    ap.add_argument("--fused", action="store_true", help="with a decode --case: the one-launch step too")
+    ap.add_argument("--train", action="store_true",
+                    help="with a prefill --case: the attention backward and the distillation signal")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -738,8 +762,15 @@ def main():
         w = Workload(args.case, torch.device("cuda", local), args.chunk)
         decode = w.c.mode == "decode"
         stage_ms, step_ms, total_ms = time_steps(w, decode, args.steps, args.warmup, None)
-        print(json.dumps({"case": w.c.name, "num_q": w.c.num_q, "ms_per_step": total_ms / args.steps,
-                          "stages_ms": stage_ms}))
+        res = {"case": w.c.name, "num_q": w.c.num_q, "ms_per_step": total_ms / args.steps,
+               "stages_ms": stage_ms}
+        if decode and args.fused:
+            flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=w.di.q.device)
+            res["fused_step_us"], res["fused_timing"] = fused_decode_us(
+                w, max(args.steps, 1), max(args.warmup, 1), lambda: flush_buf.zero_())
+        if not decode and args.train:
+            res["training_kernels"] = training_kernels_case(w, max(args.steps, 1))
+        print(json.dumps(res))
         return
 
     dist = None
