@@ -42,6 +42,7 @@ constexpr int TC_BLK = 128;           // blocks per tile (MMA N)
 constexpr int TC_PG = TC_BLK / 16;    // pages per tile
 constexpr int TC_NST = 3;             // compressed-key stages
 constexpr int TC_SAMPLE = 32;         // every 32nd tile is sampled
+constexpr int TC_KEEP = 32;           // best sampled scores kept per half-row (threshold rank)
 constexpr int TC_EPI = 8;             // epilogue warps
 constexpr int TC_THREADS = (2 + TC_EPI) * 32;
 constexpr int TC_A_BYTES = 4 * 2 * TC_ROWS * 128;  // 4 heads x 2 K-halves x 128 rows x 128 B
@@ -132,6 +133,176 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
 __device__ __forceinline__ bool bit_of(const uint32_t* b, int i) { return (b[i >> 5] >> (i & 31)) & 1u; }
+
+// v[base + j] for a run-time j in 0..31, out of registers: a 5-level select tree (31 selects, 5
+// deep) instead of a chain of 31 dependent selects.
+__device__ __forceinline__ float pick32(const float (&v)[64], int base, int j) {
+  float l1[16], l2[8], l3[4], l4[2];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) l1[k] = (j & 1) ? v[base + 2 * k + 1] : v[base + 2 * k];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) l2[k] = (j & 2) ? l1[2 * k + 1] : l1[2 * k];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) l3[k] = (j & 4) ? l2[2 * k + 1] : l2[2 * k];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) l4[k] = (j & 8) ? l3[2 * k + 1] : l3[2 * k];
+  return (j & 16) ? l4[1] : l4[0];
+}
+
+// ------------------------------------------------------------------ final selection, one warp
+// The row's candidate keys are staged in the warp's share of the (then idle) operand memory:
+// sk[0..n0) from column half 0 and sk[n0..n0+n1) from column half 1, each list ascending by
+// block.  Shared memory keeps every pass of the select at shared-memory latency.
+constexpr int TC_SEL_REGION = (TC_A_BYTES + TC_B_BYTES) / TC_EPI;  // bytes per epilogue warp
+constexpr int TC_SEL_HIST = 256;                                  // 8-bit digits
+constexpr int TC_SEL_KEYS = (TC_SEL_REGION - TC_SEL_HIST * 4) / 8;
+static_assert(TC_SEL_REGION % 16 == 0 && TC_SEL_REGION >= 2048 * 4, "selection region");
+
+// The need-th largest of the n unique keys sk[0..n), 1 <= need <= n: MSB-first radix select with
+// 8-bit digits starting at the highest bit where the keys differ; stops as soon as the digit's
+// bucket is kept whole (its smallest key is then the answer).
+__device__ __forceinline__ u64 tc_kth_largest(const u64* sk, int n, int need, uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  u64 lo = ~0ull, hi = 0ull;
+  for (int i = lane; i < n; i += 32) {
+    const u64 k = sk[i];
+    lo = k < lo ? k : lo;
+    hi = k > hi ? k : hi;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const u64 x = __shfl_xor_sync(0xffffffffu, lo, o), y = __shfl_xor_sync(0xffffffffu, hi, o);
+    lo = x < lo ? x : lo;
+    hi = y > hi ? y : hi;
+  }
+  if (need == n) return lo;
+  if (need == 1) return hi;
+  int top = 63 - __clzll((long long)(lo ^ hi));  // lo != hi: n >= 2 unique keys
+  u64 mask = top == 63 ? 0ull : ~((2ull << top) - 1ull);
+  u64 prefix = hi & mask;
+  uint32_t remaining = (uint32_t)need;
+  for (;;) {
+    const int width = top + 1 < 8 ? top + 1 : 8;
+    const int shift = top + 1 - width;
+    const uint32_t dmask = (1u << width) - 1u;
+#pragma unroll
+    for (int j = 0; j < TC_SEL_HIST / 32; ++j) hist[j * 32 + lane] = 0;
+    __syncwarp();
+    for (int b0 = 0; b0 < n; b0 += 128) {  // four loads in flight per lane, then the atomics
+      u64 k[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = b0 + u * 32 + lane;
+        k[u] = i < n ? sk[i] : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = b0 + u * 32 + lane;
+        if (i < n && (k[u] & mask) == prefix) atomicAdd(&hist[(uint32_t)(k[u] >> shift) & dmask], 1u);
+      }
+    }
+    __syncwarp();
+    // lane l owns bins 255-8l down to 248-8l, counted from the top; the sum reads them in a
+    // lane-staggered order, so the 32 lanes hit 32 different banks
+    uint32_t tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tot += hist[255 - 8 * lane - ((j + (lane >> 2)) & 7)];
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - tot;
+    const bool mine = excl < remaining && remaining <= incl;
+    int digit = 0;
+    uint32_t above = 0, cnt_at = 0;
+    if (mine) {
+      uint32_t acc = excl;
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t c = hist[255 - 8 * lane - j];
+        if (acc + c >= remaining) {
+          digit = 255 - 8 * lane - j;
+          above = acc;
+          cnt_at = c;
+          break;
+        }
+        acc += c;
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    cnt_at = __shfl_sync(0xffffffffu, cnt_at, src);
+    remaining -= above;
+    prefix |= (u64)digit << shift;
+    mask |= (u64)dmask << shift;
+    __syncwarp();
+    if (shift == 0) return prefix;
+    if (cnt_at == remaining) {  // the whole bucket is kept: the answer is its smallest key
+      u64 m = ~0ull;
+      for (int i = lane; i < n; i += 32) {
+        const u64 k = sk[i];
+        if ((k & mask) == prefix && k < m) m = k;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const u64 x = __shfl_xor_sync(0xffffffffu, m, o);
+        m = x < m ? x : m;
+      }
+      return m;
+    }
+    top = shift - 1;
+  }
+}
+
+// Keep the keys >= kth of s[0..n), compacted in place in their order; returns how many.
+__device__ __forceinline__ int tc_keep_inplace(u64* s, int n, u64 kth) {
+  const int lane = threadIdx.x & 31;
+  int w = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const u64 k = i < n ? s[i] : 0ull;
+    const bool keep = i < n && k >= kth;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);  // every lane has read before any writes
+    if (keep) s[w + __popc(bal & ((1u << lane) - 1u))] = k;
+    w += __popc(bal);
+    __syncwarp();
+  }
+  return w;
+}
+
+// The selection row from two disjoint lists of kept keys, each ascending by block (a larger low
+// word is a smaller block): a merge path, each lane writing a contiguous run of output positions,
+// then the tail block and the padding.
+__device__ __forceinline__ void tc_write_merged(const u64* A, int na, const u64* B, int nb, int row,
+                                                int tail, const ScoreArgs& a) {
+  const int lane = threadIdx.x & 31;
+  const int n = na + nb;
+  int32_t* srow = a.sel + (long long)row * a.sel_stride;
+  float* crow = a.sel_scores ? a.sel_scores + (long long)row * a.sel_stride : nullptr;
+  auto before = [](u64 x, u64 y) { return (uint32_t)x > (uint32_t)y; };  // block(x) < block(y)
+  const int per = (n + 31) >> 5;
+  const int d0 = min(lane * per, n), d1 = min(d0 + per, n);
+  int lo = max(0, d0 - nb), hi = min(d0, na);
+  while (lo < hi) {  // how many of the first d0 outputs come from A
+    const int mid = (lo + hi) >> 1;
+    if (before(A[mid], B[d0 - mid - 1])) lo = mid + 1;
+    else hi = mid;
+  }
+  int i = lo, j = d0 - lo;
+  for (int d = d0; d < d1; ++d) {
+    const bool takeA = j >= nb || (i < na && before(A[i], B[j]));
+    const u64 k = takeA ? A[i++] : B[j++];
+    srow[d] = (int32_t)key_block(k);
+    if (crow) crow[d] = key_score(k);
+  }
+  for (int d = n + lane; d < a.sel_stride; d += 32) {
+    srow[d] = d == n ? tail : -1;
+    if (crow) crow[d] = d == n ? __int_as_float(0x7f800000) : __int_as_float(0x7fc00000);
+  }
+  if (lane == 0) a.n_sel[row] = n + 1;
+}
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
     score_tc_kernel(ScoreArgs a, const __grid_constant__ CUtensorMap tmA,
@@ -315,9 +486,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
       for (int h = 0; h < 4; ++h)
         w[h] = row0 + row < a.num_q ? __bfloat162float(a.idx_w[(long long)(row0 + row) * kHi + h]) : 0.f;
-      float top[32];
+      float top[TC_KEEP];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) top[k] = -INFINITY;
+      for (int k = 0; k < TC_KEEP; ++k) top[k] = -INFINITY;
       float mn = -INFINITY, tau = -INFINITY;
       int cnt = 0;
       u64* mybuf = cand + ((long long)(row0 + row) * 2 + hf) * TC_CAP;
@@ -377,20 +548,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           while (hits) {
             const int j = __ffs(hits) - 1;
             hits &= hits - 1;
-            float x = sc[half * 32];
-#pragma unroll
-            for (int k = 1; k < 32; ++k) x = (j == k) ? sc[half * 32 + k] : x;
+            const float x = pick32(sc, half * 32, j);
             if (x > mn) {  // replace one current minimum, then recompute the minimum
               bool done = false;
 #pragma unroll
-              for (int k = 0; k < 32; ++k) {
+              for (int k = 0; k < TC_KEEP; ++k) {
                 const bool hit = !done && top[k] == mn;
                 top[k] = hit ? x : top[k];
                 done |= hit;
               }
               mn = top[0];
 #pragma unroll
-              for (int k = 1; k < 32; ++k) mn = fminf(mn, top[k]);
+              for (int k = 1; k < TC_KEEP; ++k) mn = fminf(mn, top[k]);
             }
           }
         }
@@ -418,9 +587,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           while (hits) {  // ascending block order
             const int j = __ffs(hits) - 1;
             hits &= hits - 1;
-            float x = sc[half * 32];
-#pragma unroll
-            for (int k = 1; k < 32; ++k) x = (j == k) ? sc[half * 32 + k] : x;
+            const float x = pick32(sc, half * 32, j);
             if (cnt < TC_CAP) mybuf[cnt] = make_key(x, (uint32_t)(bbase + half * 32 + j));
             ++cnt;
           }
@@ -433,13 +600,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (warp >= 2 && !m->abort_flag) {
       // ---------------------------------------------------------------- exact final selection
       // Both half-row lists are ascending by block.  Find the need-th largest key of their union,
-      // keep the keys >= it from each list in order, and merge the two by rank.
+      // keep the keys >= it from each list in order, and merge the two by block.
       const int e = warp - 2;
-      uint32_t* hist = reinterpret_cast<uint32_t*>(sB) + e * 2048;  // 8 KB per warp
-      uint32_t* blk_a = hist;                                       // reused after the select
-      float* sc_a = reinterpret_cast<float*>(hist + 512);
-      uint32_t* blk_b = hist + 1024;
-      float* sc_b = reinterpret_cast<float*>(hist + 1536);
+      uint8_t* region = smem + e * TC_SEL_REGION;  // operand memory, idle until the next segment
+      uint32_t* hist = reinterpret_cast<uint32_t*>(region);
+      u64* sk = reinterpret_cast<u64*>(region + TC_SEL_HIST * 4);
       for (int rr = 0; rr < 16; ++rr) {
         const int row = e * 16 + rr;
         if (!bit_of(m->inseg, row)) continue;
@@ -451,14 +616,55 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           continue;
         }
         if (need == 0) {
-          write_selection(row0 + row, 0, lim, blk_a, sc_a, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
+          tc_write_merged(sk, 0, sk, 0, row0 + row, lim, a);
           __syncwarp();
           continue;
         }
-        // the candidate buffers (L2-resident) are read in place
         const u64* ka = cand + (long long)(row0 + row) * 2 * TC_CAP;
         const u64* kb = ka + TC_CAP;
-        const u64 kth = warp_kth_largest2(ka, n0, kb, n0 + n1, need, hist);
+        if (n0 + n1 <= TC_SEL_KEYS) {
+          // stage sk = ka[0..n0) ++ kb[0..n1): 16-byte loads (both lists start 16-byte aligned),
+          // two in flight per lane
+          const ulonglong2* ga = reinterpret_cast<const ulonglong2*>(ka);
+          const ulonglong2* gb = reinterpret_cast<const ulonglong2*>(kb);
+          const int pa = (n0 + 1) >> 1, pb = (n1 + 1) >> 1;
+          for (int b0 = 0; b0 < pa + pb; b0 += 64) {
+            ulonglong2 v[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int i = b0 + u * 32 + lane;
+              if (i < pa) v[u] = ga[i];
+              else if (i < pa + pb) v[u] = gb[i - pa];
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int i = b0 + u * 32 + lane;
+              if (i < pa) {
+                sk[2 * i] = v[u].x;
+                if (2 * i + 1 < n0) sk[2 * i + 1] = v[u].y;
+              } else if (i < pa + pb) {
+                const int j = i - pa;
+                sk[n0 + 2 * j] = v[u].x;
+                if (2 * j + 1 < n1) sk[n0 + 2 * j + 1] = v[u].y;
+              }
+            }
+          }
+          __syncwarp();
+          const u64 kth = tc_kth_largest(sk, n0 + n1, need, hist);
+          __syncwarp();
+          const int na = tc_keep_inplace(sk, n0, kth);
+          const int nb2 = tc_keep_inplace(sk + n0, n1, kth);
+          tc_write_merged(sk, na, sk + n0, nb2, row0 + row, lim, a);
+          __syncwarp();
+          continue;
+        }
+        // more keys than the staging area holds: select from the (L2-resident) buffers in place
+        uint32_t* h2 = reinterpret_cast<uint32_t*>(region);  // 2048 words, then the kept lists
+        uint32_t* blk_a = h2;
+        float* sc_a = reinterpret_cast<float*>(h2 + 512);
+        uint32_t* blk_b = h2 + 1024;
+        float* sc_b = reinterpret_cast<float*>(h2 + 1536);
+        const u64 kth = warp_kth_largest2(ka, n0, kb, n0 + n1, need, h2);
         __syncwarp();
         const int na = warp_keep_sorted(ka, n0, kth, blk_a, sc_a);
         const int nb2 = warp_keep_sorted(kb, n1, kth, blk_b, sc_b);
@@ -466,6 +672,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                           a.sel_scores, a.sel_stride);
         __syncwarp();
       }
+      // the next segment's TMA copies overwrite this shared memory: order these generic accesses
+      // before them
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     }
     __syncthreads();
     if (tid < 4) m->done[tid] |= m->inseg[tid];

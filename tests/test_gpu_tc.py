@@ -90,6 +90,23 @@ def test_tc_sampled_threshold_generator_weights_exact():
     assert 0 < settled < len(rows)
 
 
+KEEP_ALL_EDGE = Config("tc_keepall_chunk4096_ctx16384", "prefill", 1, 16384, 4096, 8, 2, 64, 4, 128,
+                       shuffle_pages=True, seed=0x7C05)
+
+
+def test_tc_keep_all_rows_on_both_sides_of_the_staging_limit():
+    """Rows of 3,072-4,095 candidates keep every key.  The final select stages a row's keys in
+    shared memory when they fit (3,456 keys) and reads them in place otherwise: rows on both
+    sides of that limit, every row bit-exact and settled by the tensor-core kernel."""
+    run, w = run_positive_weights(KEEP_ALL_EDGE)
+    _, q_pos = host(KEEP_ALL_EDGE, True).rows()
+    lim = q_pos // 4
+    assert (lim <= 3456).any() and (lim > 3456).any()
+    settled = check_rows(run, range(KEEP_ALL_EDGE.num_q), True, w_bits=w, model=True)
+    assert settled == KEEP_ALL_EDGE.num_q
+    assert run.runner.error_bits() == 0
+
+
 def test_tc_c2_integer_sampled_rows():
     """The C2 chunk (16,384 tokens at 131,072) on integer inputs with positive weights: 256 rows
     across the chunk bit-exact, each settled by the tensor-core kernel, and no row of the chunk
