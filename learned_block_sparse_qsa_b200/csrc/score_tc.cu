@@ -19,16 +19,19 @@
 //               the 128 columns; thread = (query row, column half).  The weighted ReLU sum of pair
 //               X stays in registers while pair Y is computed, then X and Y are released in turn.
 // Selection without in-loop compaction: the tile sequence is first every 32nd tile (a sample),
-// then all tiles.  During the sample each thread keeps the 32 best sampled scores of its half-row
-// in registers; the row threshold tau = min over its two halves of the 32nd best, so about 2,048
-// of the row's scores are >= tau, and fewer than 512 is a ~6-sigma event.  Rows of at most
-// 2 * TC_CAP candidates skip the threshold and keep every key (a sample of one or two tiles
-// would keep too few).  The full pass appends every (score >= tau, block) key to a
-// per-half-row buffer (in ascending block order); the final step checks that at least
-// min(512, t/4) keys were kept -- which proves every true top-512 key was kept -- and selects
-// exactly (radix select on 64-bit keys, lower block index wins ties) with a merge by rank.  Rows
-// that fail the check (adversarial score orders) or overflow the buffer are recomputed by the exact
-// streaming kernel, so the result never depends on the sample.
+// then all tiles.  During the sample each thread keeps the TC_KEEP = 24 best sampled scores of
+// its half-row in registers; the row threshold tau = min over its two halves of the 24th best, so
+// about 1,700 of the row's scores are >= tau (on independent scores: mean 1,711-1,727, standard
+// deviation 260-274 at 32K-262K candidates) and fewer than 512 is a more than 4-sigma event.  Each
+// kept key costs an append and a share of the final select, so a lower rank is faster until the
+// exact fallback starts to be needed.  Rows of at most 2 * TC_CAP candidates skip the threshold
+// and keep every key (a sample of one or two tiles would keep too few).  The full pass appends
+// every (score >= tau, block) key to a per-half-row buffer (in ascending block order); the final
+// step checks that at least min(512, t/4) keys were kept -- which proves every true top-512 key
+// was kept -- and selects exactly (radix select on 64-bit keys, lower block index wins ties) and
+// merges the two lists by block.  Rows that fail the check (adversarial score orders) or overflow
+// the buffer are recomputed by the exact streaming kernel, so the result never depends on the
+// sample.
 #include "common.cuh"
 #include "internal.h"
 #include "score_common.cuh"
@@ -42,7 +45,7 @@ constexpr int TC_BLK = 128;           // blocks per tile (MMA N)
 constexpr int TC_PG = TC_BLK / 16;    // pages per tile
 constexpr int TC_NST = 3;             // compressed-key stages
 constexpr int TC_SAMPLE = 32;         // every 32nd tile is sampled
-constexpr int TC_KEEP = 32;           // best sampled scores kept per half-row (threshold rank)
+constexpr int TC_KEEP = 24;           // best sampled scores kept per half-row (threshold rank)
 constexpr int TC_EPI = 8;             // epilogue warps
 constexpr int TC_THREADS = (2 + TC_EPI) * 32;
 constexpr int TC_A_BYTES = 4 * 2 * TC_ROWS * 128;  // 4 heads x 2 K-halves x 128 rows x 128 B
@@ -53,6 +56,7 @@ constexpr int TC_CAP = 2048;          // candidate slots per half-row
 struct TcMisc {
   // tfull/tempty[0]: TMEM pair X (heads 0, 1); [1]: pair Y (heads 2, 3)
   uint64_t full[TC_NST], empty[TC_NST], tfull[2], tempty[2], aload, mma_done;
+  uint64_t stage[TC_EPI];  // final select: bulk copies of one row's candidate keys, per warp
   uint32_t tmem_base;
   int abort_flag;
   int issued, consumed;  // B tiles issued by the producer / waited for by the MMA issuer
@@ -331,6 +335,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     mbar_init(&m->aload, 1);
     mbar_init(&m->mma_done, 1);
+    for (int e = 0; e < TC_EPI; ++e) mbar_init(&m->stage[e], 1);
     m->abort_flag = 0;
     m->issued = 0;
     m->consumed = 0;
@@ -362,6 +367,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         write_empty_selection(row0 + r, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
   }
 
+  uint32_t stage_phase = 0;  // epilogue warps: phase of this warp's staging barrier
+  bool stage_dead = false;   // a staging copy never landed: the warp's remaining rows go to redo
   int it_base = 0;  // tiles of earlier segments (all roles count the same tiles)
   int segi = 0;     // segments started (phase of the query-tile barrier)
   for (;;) {
@@ -532,7 +539,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         return true;
       };
-      // -- sample tiles: keep the 32 best scores of this half-row in registers.  The hot loop is
+      // -- sample tiles: keep the TC_KEEP best scores of this half-row in registers.  The hot loop is
       // branch-free (bit masks of blocks above the current minimum); the rare insertions run from
       // one copy of the replacement code.
       for (int i = 0; i < nsamp && i < L; ++i) {
@@ -594,6 +601,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       m->cnt[hf][row] = cnt;
+      // the final select reads the candidate buffers with bulk copies (async proxy)
+      asm volatile("fence.proxy.async.global;\n" ::: "memory");
     }
     __syncthreads();  // the segment's tiles are all consumed; stage memory is free
 
@@ -622,39 +631,38 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         const u64* ka = cand + (long long)(row0 + row) * 2 * TC_CAP;
         const u64* kb = ka + TC_CAP;
-        if (n0 + n1 <= TC_SEL_KEYS) {
-          // stage sk = ka[0..n0) ++ kb[0..n1): 16-byte loads (both lists start 16-byte aligned),
-          // two in flight per lane
-          const ulonglong2* ga = reinterpret_cast<const ulonglong2*>(ka);
-          const ulonglong2* gb = reinterpret_cast<const ulonglong2*>(kb);
-          const int pa = (n0 + 1) >> 1, pb = (n1 + 1) >> 1;
-          for (int b0 = 0; b0 < pa + pb; b0 += 64) {
-            ulonglong2 v[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int i = b0 + u * 32 + lane;
-              if (i < pa) v[u] = ga[i];
-              else if (i < pa + pb) v[u] = gb[i - pa];
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int i = b0 + u * 32 + lane;
-              if (i < pa) {
-                sk[2 * i] = v[u].x;
-                if (2 * i + 1 < n0) sk[2 * i + 1] = v[u].y;
-              } else if (i < pa + pb) {
-                const int j = i - pa;
-                sk[n0 + 2 * j] = v[u].x;
-                if (2 * j + 1 < n1) sk[n0 + 2 * j + 1] = v[u].y;
-              }
-            }
+        const int n0r = (n0 + 1) & ~1, n1r = (n1 + 1) & ~1;  // 16-byte multiples
+        if (n0r + n1r <= TC_SEL_KEYS) {
+          if (stage_dead) {
+            if (lane == 0) redo[row0 + row] = 1;
+            continue;
           }
+          // stage sk = ka[0..n0) ++ [0 if n0 is odd] ++ kb[0..n1) with two bulk copies (both
+          // lists start 16-byte aligned; a copy may read one stale key past a list's end, which
+          // lies inside its buffer and is overwritten below)
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // after this warp's
+          __syncwarp();                                                    // last use of sk
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&m->stage[e], (uint32_t)(n0r + n1r) * 8u);
+            if (n0r) bulk_g2s(smem_addr(sk), ka, (uint32_t)n0r * 8u, &m->stage[e]);
+            if (n1r) bulk_g2s(smem_addr(sk + n0r), kb, (uint32_t)n1r * 8u, &m->stage[e]);
+          }
+          const bool landed = mbar_wait(&m->stage[e], stage_phase, a.err) ||
+                              mbar_wait(&m->stage[e], stage_phase, a.err);  // bounded; 2nd: drain
+          stage_phase ^= 1u;
+          if (!landed) {  // (error flagged) the row goes to the exact kernel
+            stage_dead = true;
+            if (lane == 0) redo[row0 + row] = 1;
+            continue;
+          }
+          if (lane == 0 && (n0 & 1)) sk[n0] = 0ull;  // below every key: never selected
           __syncwarp();
-          const u64 kth = tc_kth_largest(sk, n0 + n1, need, hist);
+          const int n = n0r + n1;
+          const u64 kth = tc_kth_largest(sk, n, need, hist);
           __syncwarp();
           const int na = tc_keep_inplace(sk, n0, kth);
-          const int nb2 = tc_keep_inplace(sk + n0, n1, kth);
-          tc_write_merged(sk, na, sk + n0, nb2, row0 + row, lim, a);
+          const int nb2 = tc_keep_inplace(sk + n0r, n1, kth);
+          tc_write_merged(sk, na, sk + n0r, nb2, row0 + row, lim, a);
           __syncwarp();
           continue;
         }

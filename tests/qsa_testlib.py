@@ -150,13 +150,16 @@ def positive_int_weights(w_bits: np.ndarray) -> np.ndarray:
     return orc.f64_to_bf16_bits(np.abs(w) % 3 + 1)
 
 
+TC_KEEP = 24  # the tensor-core kernel's threshold rank: best sampled scores kept per half-row
+
+
 def tc_redo_model(scores: np.ndarray, topk: int, nsamp: int, cap: int = 2048, tile: int = 128,
-                  sample_every: int = 32) -> bool:
+                  sample_every: int = 32, keep: int = TC_KEEP) -> bool:
     """Whether the tensor-core indexer kernel hands a row to the exact streaming kernel, for a row
     whose fp32 candidate scores are known exactly (integer inputs).  A model of the kernel's
     branch, not of the method: each row is split into two column halves of every 128-block tile;
     rows of more than 2 * cap candidates (and more than topk) take as threshold the smaller of the
-    two halves' 32nd-best score over the sampled tiles (tiles 0, 32, ..., 32 * (nsamp - 1));
+    two halves' keep-th best score over the sampled tiles (tiles 0, 32, ..., 32 * (nsamp - 1));
     every key at or above it is kept; the row is redone when a half keeps more than cap keys or
     the row keeps fewer than min(topk, candidates)."""
     lim = scores.shape[0]
@@ -170,7 +173,7 @@ def tc_redo_model(scores: np.ndarray, topk: int, nsamp: int, cap: int = 2048, ti
         thr = []
         for hf in (0, 1):
             v = np.sort(scores[sampled & (half == hf)])[::-1]
-            thr.append(v[31] if v.size >= 32 else -np.inf)
+            thr.append(v[keep - 1] if v.size >= keep else -np.inf)
         tau = min(thr)
     keep = scores >= tau
     n0, n1 = int(np.sum(keep & (half == 0))), int(np.sum(keep & (half == 1)))

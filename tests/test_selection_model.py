@@ -171,14 +171,14 @@ def test_short_rows_keep_every_candidate():
 # --------------------------------------------------------------------------------------------
 # The prefill indexer's sampled threshold.  The tile sequence is first every 32nd tile of 128
 # blocks (the sample), then all tiles.  Each half-row (blocks 64h..64h+63 of every tile) keeps its
-# 32 best sampled scores.  The row threshold is the smaller of the two halves' 32nd best (minus
+# 24 best sampled scores.  The row threshold is the smaller of the two halves' 24th best (minus
 # infinity when the row has no more candidates than the budget or than the two half-row buffers
-# hold, or when a half sampled fewer than 32).
+# hold, or when a half sampled fewer than 24).
 # Every key at or above it is kept, and the exact select runs over the kept keys.  The row is
 # handed to the exact path when fewer than need keys were kept, or a half-row kept more than its
 # 2,048 slots.
 
-TILE, SAMPLE_EVERY, SAMPLE_KEEP, HALF_CAP = 128, 32, 32, 2048
+TILE, SAMPLE_EVERY, SAMPLE_KEEP, HALF_CAP = 128, 32, 24, 2048
 
 
 def sampled_select(scores32: np.ndarray, topk: int = 512):
