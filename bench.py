@@ -157,14 +157,15 @@ def traffic_for(kernel_file: str, key: str):
         return None
     if not d:
         return None
-    src = os.path.join(ROOT, "learned_block_sparse_qsa_b200", "csrc", kernel_file)
-    return d["bytes_per_launch"] if d.get("source_sha") == code_sha(src) else None
+    files = kernel_file if isinstance(kernel_file, (list, tuple)) else [kernel_file]
+    srcs = [os.path.join(ROOT, "learned_block_sparse_qsa_b200", "csrc", f) for f in files]
+    return d["bytes_per_launch"] if d.get("source_sha") == code_sha(*srcs) else None
 
 
-def code_sha(path: str) -> str:
-    """Hash of a CUDA source with comments and blank space removed: counters stay attached to
+def code_sha(*paths: str) -> str:
+    """Hash of CUDA sources with comments and blank space removed: counters stay attached to
     the code they were taken on, and an edit of a comment does not orphan them."""
-    text = open(path, encoding="utf-8").read()
+    text = "\n".join(open(p, encoding="utf-8").read() for p in paths)
     text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
     text = re.sub(r"//[^\n]*", " ", text)
     text = " ".join(text.split())
@@ -814,7 +815,7 @@ def main():
                            peak=peaks["tf"], kernel_file="score_tc.cu"),
         "sparse_attn": dict(ms=stage_ms["sparse_attn"], bound="hbm", unit="GB/s",
                             achieved=work["attn_bytes"] / (stage_ms["sparse_attn"] * 1e-3) / 1e9,
-                            peak=peaks["hbm"], kernel_file="attn.cu"),
+                            peak=peaks["hbm"], kernel_file=("attn.cu", "attn_sw.cuh")),
     }
     for s in stages.values():
         s["frac"] = s["achieved"] / s["peak"]
