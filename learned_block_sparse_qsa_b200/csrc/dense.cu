@@ -5,6 +5,8 @@
 // attention at one million tokens.  This kernel is that baseline on the same paged pools, so the
 // sparse/dense ratio measured here compares two kernels of this library.
 //
+// The prefill form at head_dim 128 runs on the tensor cores (dense_tc.cu); this file holds the
+// mma.sync kernel for the other shapes and the decode form.
 // Flash-attention tiling: a CTA owns MR = TQ x G query rows of one KV head (the G query heads of
 // TQ consecutive tokens of one sequence), streams the sequence's pages (64 positions) of that KV
 // head through a 3-stage cp.async ring, and keeps fp32 online-softmax state in registers.  The
@@ -333,6 +335,7 @@ cudaError_t launch_dense_attn(const Geometry& g, const void* q, const void* k_po
                               const void* v_pool, void* out, float* lse, int splits, void* ws,
                               cudaStream_t s) {
   if (g.num_q == 0) return cudaSuccess;
+  if (splits == 1 && dense_tc_supported(g)) return launch_dense_tc(g, q, k_pool, v_pool, out, lse, s);
   DenseArgs a;
   a.q = static_cast<const bf16*>(q);
   a.k_pool = static_cast<const bf16*>(k_pool);

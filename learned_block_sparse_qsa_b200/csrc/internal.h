@@ -53,6 +53,10 @@ cudaError_t launch_sparse_attn(const Geometry& g, const void* q, const void* k_p
 
 // dense.cu
 int resolve_dense_splits(const Geometry& g, int requested);
+// dense_tc.cu: the prefill form on tcgen05 (head_dim 128, 128 % G == 0, tensor maps available)
+bool dense_tc_supported(const Geometry& g);
+cudaError_t launch_dense_tc(const Geometry& g, const void* q, const void* k_pool, const void* v_pool,
+                            void* out, float* lse, cudaStream_t s);
 size_t dense_decode_workspace_bytes(const Geometry& g, int splits);
 cudaError_t launch_dense_attn(const Geometry& g, const void* q, const void* k_pool,
                               const void* v_pool, void* out, float* lse, int splits, void* ws,

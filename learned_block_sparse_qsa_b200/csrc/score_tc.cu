@@ -36,6 +36,7 @@
 #include "internal.h"
 #include "score_common.cuh"
 #include "select.cuh"
+#include "tc_common.cuh"
 
 namespace qsa {
 namespace {
@@ -71,17 +72,8 @@ struct TcMisc {
 constexpr int TC_SMEM = TC_A_BYTES + TC_B_BYTES + (int)((sizeof(TcMisc) + 127) / 128 * 128);
 static_assert(TC_SMEM <= 232448, "shared memory budget");
 
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
-  uint64_t d = (uint64_t)((addr >> 4) & 0x3FFF);
-  d |= (uint64_t)1 << 16;            // leading byte offset (unused with the 128-byte swizzle)
-  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: 8 rows x 128 B
-  d |= (uint64_t)1 << 46;            // descriptor version
-  d |= (uint64_t)2 << 61;            // 128-byte swizzle
-  return d;
-}
 // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M=128, N=128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_BLK >> 3) << 17) |
-                            ((uint32_t)(TC_ROWS >> 4) << 24);
+constexpr uint32_t kIdesc = idesc_bf16(TC_ROWS, TC_BLK, false);
 
 // Packed fp32 pairs (sm_100): one instruction rounds both lanes exactly as the scalar op would.
 __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
@@ -108,33 +100,7 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   return r;
 }
 
-__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                   smem_addr(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(TC_EPI * 32)); }
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
 __device__ __forceinline__ bool bit_of(const uint32_t* b, int i) { return (b[i >> 5] >> (i & 31)) & 1u; }
 
@@ -473,13 +439,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t ad = sw128_desc(ast + (ks >> 2) * (TC_ROWS * 128) + (ks & 3) * 32);
                 const uint64_t bd = sw128_desc(bst + (ks >> 2) * (TC_BLK * 128) + (ks & 3) * 32);
-                mma_f16(tbase + pair * 256 + hh * TC_BLK, ad, bd, ks > 0 ? 1u : 0u);
+                umma_bf16(tbase + pair * 256 + hh * TC_BLK, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
               }
             }
-            mma_commit(&m->tfull[pair]);
+            umma_commit(&m->tfull[pair]);
           }
           if (!ok) break;
-          mma_commit(&m->empty[s]);
+          umma_commit(&m->empty[s]);
         }
         if (!ok) m->abort_flag = 1;
       }
@@ -699,7 +665,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
   if (warp == 1) {
     if (lane == 0 && it_base > 0) {  // every issued MMA has completed before TMEM is released
-      mma_commit(&m->mma_done);
+      umma_commit(&m->mma_done);
       mbar_wait(&m->mma_done, 0, a.err);
     }
     __syncwarp();
