@@ -5,18 +5,22 @@
 // three different experiments": the QSA module's speedups are quoted against paged grouped-query
 // attention.  This is that baseline on the same paged pools (head_dim 128).
 //
-// CTA = M = 128 rows: TQ = 128 / G consecutive tokens x the G query heads of one KV head (row =
-// token * G + head), warp-specialised:
-//   warp 0      TMA producer: the CTA's query tile once (32 KB), then K and V tiles of 128
+// CTA = two query tiles (A and B) of M = 128 rows each, sharing every K/V tile: a tile's 64 KB
+// of keys and values feeds 2 x 8.4 MFLOP.  A query tile is TQ = 128 / G consecutive tokens x the G
+// query heads of one KV head (row = token * G + head).  Warp-specialised:
+//   warp 0      TMA producer: the two query tiles once (64 KB), then K and V tiles of 128
 //               positions (two 64-token pages) of the KV head into a 2-stage ring (64 KB each);
-//   warp 1      owns the tensor memory (S0 | S1 | O, 128 columns each) and one lane issues, per
-//               tile j, S_j = Q K_j^T into S[j % 2] and then O += P_{j-1} V_{j-1} for the
-//               previous tile (P from shared memory, V as an MN-major operand), so that the
-//               softmax of one tile overlaps the MMAs of its neighbours;
-//   warps 2-5   softmax, one row per thread: read S_j, mask positions after t, scale to base 2,
-//               keep the row's reference maximum (raised, with O and the running sum rescaled,
-//               only when a tile's maximum exceeds it by more than 8: lazy rescaling), write
-//               P_j = 2^(s - m) as bf16 into shared memory; at the end O / l and the log-sum-exp.
+//   warp 1      owns the tensor memory (per query tile: S/P 128 columns, O 128 columns) and one
+//               lane issues, per query tile q and K/V tile j: O_q += P_q(j) V_j (P read from
+//               tensor memory, V as an MN-major operand), then S_q(j+1) = Q_q K_{j+1}^T into the
+//               same columns that held S_q(j) and P_q(j) (MMAs of one thread run in issue order);
+//               the two query tiles alternate, so that one tile's softmax overlaps the other's MMAs;
+//   warps 2-5 / 6-9  softmax of query tile A / B, one row per thread: two reads of S_q(j) (the
+//               row maximum, then the exponentials), mask positions after t, keep the row's
+//               reference maximum in base 2 (raised, with O and the running sum rescaled, only when
+//               a tile's maximum exceeds it by more than 8: lazy rescaling), and write
+//               P = 2^(scale * s - m) as bf16 pairs over the tile's own S columns; at the end
+//               O / l and the log-sum-exp.
 // Rows of a CTA that belong to different sequences are handled one sequence (segment) at a time.
 // Cache slots after a segment's last position may be unwritten: their V rows are zeroed in the
 // last tile before the MMA reads them, so a masked probability (0) never meets a non-finite value.
@@ -28,33 +32,32 @@
 namespace qsa {
 namespace {
 
-constexpr int DT_ROWS = 128;  // MMA M
+constexpr int DT_ROWS = 128;  // MMA M (one query tile)
+constexpr int DT_NQ = 2;      // query tiles per CTA
 constexpr int DT_POS = 128;   // positions per K/V tile: N of S, K of P V
 constexpr int DT_NST = 2;     // K/V stages
-constexpr int DT_SMW = 4;     // softmax warps
-constexpr int DT_THREADS = (2 + DT_SMW) * 32;
+constexpr int DT_SMW = 4;     // softmax warps per query tile
+constexpr int DT_THREADS = (2 + DT_NQ * DT_SMW) * 32;
 constexpr int DT_HALF = DT_ROWS * 128;         // one 64-column (128-byte) half of a 128-row tile
-constexpr int DT_Q_BYTES = 2 * DT_HALF;        // query tile, K-major: [k-half][row][128 B]
+constexpr int DT_Q_BYTES = 2 * DT_HALF;        // one query tile, K-major: [k-half][row][128 B]
 constexpr int DT_KV_BYTES = 2 * DT_HALF;       // K tile [k-half][position][128 B];
                                                // V tile [page][dim-half][64 positions][128 B]
 constexpr int DT_STAGE = 2 * DT_KV_BYTES;      // K + V
-constexpr int DT_P_BYTES = 2 * DT_HALF;        // P tile, K-major: [position-half][row][128 B]
 constexpr float DT_RESCALE = 8.f;              // lazy rescaling threshold (base-2 exponent)
 constexpr uint32_t kIdescS = idesc_bf16(DT_ROWS, DT_POS, false);
 constexpr uint32_t kIdescPV = idesc_bf16(DT_ROWS, 128, true);
 
 struct DtMisc {
-  uint64_t qload, kv_full[DT_NST], kv_empty[DT_NST], s_full[2], s_empty[2], p_full[2], p_empty[2];
+  uint64_t qload, kv_full[DT_NST], kv_empty[DT_NST], s_full[DT_NQ], p_full[DT_NQ], o_done[DT_NQ];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
   int issued, consumed;  // K/V tiles issued by the producer / waited for by the MMA issuer
   int seg, tmax, ntile;
-  uint32_t done[4];   // tokens already handled (bit per token)
-  uint32_t inseg[4];  // tokens of the current segment
+  uint32_t done[8];   // tokens already handled (bit per token)
+  uint32_t inseg[8];  // tokens of the current segment
 };
-constexpr int DT_SMEM = DT_Q_BYTES + DT_NST * DT_STAGE + 2 * DT_P_BYTES +
-                        (int)((sizeof(DtMisc) + 127) / 128 * 128);
+constexpr int DT_SMEM = DT_NQ * DT_Q_BYTES + DT_NST * DT_STAGE + (int)((sizeof(DtMisc) + 127) / 128 * 128);
 static_assert(DT_SMEM <= 232448, "shared memory budget");
 
 struct DtArgs {
@@ -82,12 +85,12 @@ __global__ void __launch_bounds__(DT_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + DT_Q_BYTES;
-  uint8_t* sP = sKV + DT_NST * DT_STAGE;
-  DtMisc* m = reinterpret_cast<DtMisc*>(sP + 2 * DT_P_BYTES);
+  uint8_t* sKV = smem + DT_NQ * DT_Q_BYTES;
+  DtMisc* m = reinterpret_cast<DtMisc*>(sKV + DT_NST * DT_STAGE);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int TQ = a.TQ, G = a.G;
-  const int tok0 = blockIdx.x * TQ;
+  const int NT = DT_NQ * TQ;  // tokens of the CTA
+  const int tok0 = blockIdx.x * NT;
   const int g = blockIdx.y;
 
   if (smem_addr(smem) & 1023) {  // operand tiles need 1024-byte alignment
@@ -100,19 +103,18 @@ __global__ void __launch_bounds__(DT_THREADS, 1)
       mbar_init(&m->kv_full[s], 1);
       mbar_init(&m->kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&m->s_full[b], 1);
-      mbar_init(&m->s_empty[b], DT_SMW);
-      mbar_init(&m->p_full[b], DT_SMW);
-      mbar_init(&m->p_empty[b], 1);
+    for (int q = 0; q < DT_NQ; ++q) {
+      mbar_init(&m->s_full[q], 1);
+      mbar_init(&m->p_full[q], DT_SMW);
+      mbar_init(&m->o_done[q], 1);
     }
     mbar_init(&m->mma_done, 1);
     m->abort_flag = 0;
     m->issued = 0;
     m->consumed = 0;
-    for (int i = 0; i < 4; ++i) m->done[i] = 0;
+    for (int i = 0; i < 8; ++i) m->done[i] = 0;
     // tokens that fail validation are done from the start (their rows are never written)
-    for (int i = 0; i < TQ; ++i) {
+    for (int i = 0; i < NT; ++i) {
       const int r = tok0 + i;
       bool bad = r >= a.num_q;
       if (!bad) {
@@ -136,23 +138,26 @@ __global__ void __launch_bounds__(DT_THREADS, 1)
   tc_fence_after();
   const uint32_t tbase = m->tmem_base;
 
-  if (warp == 0 && lane == 0) {  // the query tile, once: rows past num_q read as zeros
-    mbar_arrive_expect_tx(&m->qload, DT_Q_BYTES);
-    for (int kh = 0; kh < 2; ++kh) tma3d(smem_addr(sQ + kh * DT_HALF), &tmQ, kh * 64, g * G, tok0, &m->qload);
+  if (warp == 0 && lane == 0) {  // the query tiles, once: rows past num_q read as zeros
+    mbar_arrive_expect_tx(&m->qload, DT_NQ * DT_Q_BYTES);
+    for (int q = 0; q < DT_NQ; ++q)
+      for (int kh = 0; kh < 2; ++kh)
+        tma3d(smem_addr(sQ + q * DT_Q_BYTES + kh * DT_HALF), &tmQ, kh * 64, g * G, tok0 + q * TQ, &m->qload);
   }
 
-  // softmax thread's row: TMEM lane quarter warp % 4
+  // softmax thread: query tile qt, row (TMEM lane quarter warp % 4)
+  const int qt = warp >= 2 ? (warp - 2) / DT_SMW : 0;
   const int row = 32 * (warp & 3) + lane;
-  const int tok = row / G, head = row % G;
-  float m_ref = -INFINITY, l_sum = 0.f;
+  const int tok = qt * TQ + row / G, head = row % G;
+  const uint32_t tS = tbase + qt * 256, tO = tS + 128;  // this query tile's S/P and O columns
 
   int gbase = 0;  // tiles of earlier segments (every role counts the same tiles)
   for (;;) {
     __syncthreads();
     if (tid == 0) {  // next segment: the sequence of the first token not yet done
       int seg = -1, tmax = -1;
-      for (int i = 0; i < 4; ++i) m->inseg[i] = 0;
-      for (int i = 0; i < TQ; ++i) {
+      for (int i = 0; i < 8; ++i) m->inseg[i] = 0;
+      for (int i = 0; i < NT; ++i) {
         if (dt_bit(m->done, i)) continue;
         const int s = a.q_seq[tok0 + i];
         if (seg < 0) seg = s;
@@ -210,151 +215,149 @@ __global__ void __launch_bounds__(DT_THREADS, 1)
       // ---------------------------------------------------------------- MMA issuer
       if (lane == 0) {
         bool ok = gbase > 0 || mbar_wait(&m->qload, 0, a.err);
-        auto pv = [&](int jp) -> bool {  // O (+)= P_jp V_jp
-          const int gp = gbase + jp, bp = gp & 1, sp = gp % DT_NST;
-          if (!mbar_wait(&m->p_full[bp], (gp >> 1) & 1, a.err)) return false;
-          tc_fence_after();
-          const uint32_t pa = smem_addr(sP + bp * DT_P_BYTES);
-          const uint32_t vb = smem_addr(sKV + sp * DT_STAGE + DT_KV_BYTES);
-#pragma unroll
-          for (int ks = 0; ks < DT_POS / 16; ++ks) {
-            const uint64_t ad = sw128_desc(pa + (ks >> 2) * DT_HALF + (ks & 3) * 32);
-            const uint64_t bd = sw128_desc_mn(vb + (ks >> 2) * DT_HALF + (ks & 3) * 2048, DT_HALF / 2);
-            umma_bf16(tbase + 256, ad, bd, kIdescPV, (jp > 0 || ks > 0) ? 1u : 0u);
-          }
-          umma_commit(&m->p_empty[bp]);
-          umma_commit(&m->kv_empty[sp]);
-          return true;
-        };
-        for (int j = 0; ok && j < ntile; ++j) {
-          const int gj = gbase + j, s = gj % DT_NST, b = gj & 1;
-          if (!mbar_wait(&m->kv_full[s], (gj / DT_NST) & 1, a.err)) { ok = false; break; }
-          m->consumed = gj + 1;
-          if (gj >= 2 && !mbar_wait(&m->s_empty[b], ((gj >> 1) & 1) ^ 1, a.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t qa = smem_addr(sQ), kb = smem_addr(sKV + s * DT_STAGE);
+        auto s_mma = [&](int q, int j) {  // S_q(j) = Q_q K_j^T
+          const uint32_t qa = smem_addr(sQ + q * DT_Q_BYTES);
+          const uint32_t kb = smem_addr(sKV + ((gbase + j) % DT_NST) * DT_STAGE);
 #pragma unroll
           for (int ks = 0; ks < 128 / 16; ++ks) {
             const uint64_t ad = sw128_desc(qa + (ks >> 2) * DT_HALF + (ks & 3) * 32);
             const uint64_t bd = sw128_desc(kb + (ks >> 2) * DT_HALF + (ks & 3) * 32);
-            umma_bf16(tbase + b * 128, ad, bd, kIdescS, ks > 0 ? 1u : 0u);
+            umma_bf16(tbase + q * 256, ad, bd, kIdescS, ks > 0 ? 1u : 0u);
           }
-          umma_commit(&m->s_full[b]);
-          if (j >= 1 && !pv(j - 1)) { ok = false; break; }
+          umma_commit(&m->s_full[q]);
+        };
+        auto load_ready = [&](int j) -> bool {
+          const int gj = gbase + j;
+          if (!mbar_wait(&m->kv_full[gj % DT_NST], (gj / DT_NST) & 1, a.err)) return false;
+          m->consumed = gj + 1;
+          tc_fence_after();
+          return true;
+        };
+        if (ok && load_ready(0))
+          for (int q = 0; q < DT_NQ; ++q) s_mma(q, 0);
+        else
+          ok = false;
+        for (int j = 0; ok && j < ntile; ++j) {
+          const int gj = gbase + j;
+          const uint32_t vb = smem_addr(sKV + (gj % DT_NST) * DT_STAGE + DT_KV_BYTES);
+          for (int q = 0; ok && q < DT_NQ; ++q) {
+            if (!mbar_wait(&m->p_full[q], gj & 1, a.err)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < DT_POS / 16; ++ks) {  // O_q (+)= P_q(j) V_j
+              const uint64_t bd = sw128_desc_mn(vb + (ks >> 2) * DT_HALF + (ks & 3) * 2048, DT_HALF / 2);
+              umma_bf16_ts(tbase + q * 256 + 128, tbase + q * 256 + ks * 8, bd, kIdescPV,
+                           (j > 0 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(&m->o_done[q]);
+            if (j + 1 < ntile) {
+              if (q == 0 && !load_ready(j + 1)) { ok = false; break; }
+              s_mma(q, j + 1);  // overwrites S_q(j) / P_q(j): after the PV above, in issue order
+            }
+          }
+          if (ok) umma_commit(&m->kv_empty[gj % DT_NST]);
         }
-        if (ok && ntile > 0) ok = pv(ntile - 1);
         if (!ok) m->abort_flag = 1;
       }
     } else {
       // ---------------------------------------------------------------- softmax
-      const bool act = tok < TQ && dt_bit(m->inseg, tok);
+      const bool act = dt_bit(m->inseg, tok);
       const int t = act ? a.q_pos[tok0 + tok] : -1;
-      const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-      m_ref = -INFINITY;
-      l_sum = 0.f;
+      const uint32_t lb = (uint32_t)(32 * (warp & 3)) << 16;  // TMEM lane base of this warp
+      float m_ref = -INFINITY, l_sum = 0.f;
+      // A warp that gives up waiting (error flagged) goes on without its waits and tensor-memory
+      // accesses, with `dead` warp-uniform, so that the collective accesses stay uniform.
       bool dead = false;
-      for (int j = 0; j < ntile && !dead; ++j) {
-        const int gj = gbase + j, b = gj & 1, s = gj % DT_NST;
-        const int P0 = j * DT_POS;
-        if (!mbar_wait(&m->s_full[b], (gj >> 1) & 1, a.err)) {
+      auto waitw = [&](uint64_t* bar, uint32_t par) {
+        if (dead) return;
+        const bool okw = mbar_wait(bar, par, a.err);
+        if (__any_sync(0xffffffffu, !okw)) {
           m->abort_flag = 1;
           dead = true;
-          break;
         }
-        tc_fence_after();
-        float v[DT_POS];
+      };
+      for (int j = 0; j < ntile; ++j) {
+        const int gj = gbase + j, s = gj % DT_NST;
+        const int P0 = j * DT_POS;
+        // S_q(j) is complete, and with it every earlier MMA (P_q(j-1) has been read, O_q holds
+        // tiles < j)
+        waitw(&m->s_full[qt], gj & 1);
+        const bool vis = P0 + DT_POS - 1 <= t;  // whole tile visible: no mask
+        // pass 1: the row maximum
+        float mx[8];
 #pragma unroll
-        for (int c = 0; c < DT_POS / 16; ++c) {
-          float x[16];
-          tmem_ld16(tbase + lane_base + b * 128 + c * 16, x);
+        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+        if (!dead) {
+          tc_fence_after();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[c * 16 + e] = x[e];
+          for (int c = 0; c < DT_POS / 16; ++c) {
+            float x[16];
+            tmem_ld16(tS + lb + c * 16, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float y = (vis || P0 + c * 16 + e <= t) ? x[e] : -INFINITY;
+              mx[e & 7] = fmaxf(mx[e & 7], y);
+            }
+          }
         }
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&m->s_empty[b]);
-        // mask positions after t (whole tile visible: no mask); the scale to base 2 is folded into
-        // the exponent below (scale > 0, so the raw maximum scales with it)
-        if (P0 + DT_POS - 1 > t) {
-#pragma unroll
-          for (int c = 0; c < DT_POS; ++c) v[c] = P0 + c <= t ? v[c] : -INFINITY;
-        }
-        float mx[8];  // maximum as a tree: 8 independent chains, then 3 levels
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = v[e];
-#pragma unroll
-        for (int c = 8; c < DT_POS; c += 8)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], v[c + e]);
         const float tmx = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * a.scale_log2;
         const float m_new = fmaxf(m_ref, tmx);
         const bool resc = m_ref != -INFINITY && m_new > m_ref + DT_RESCALE;
-        if (__any_sync(0xffffffffu, resc)) {
-          // O holds tiles < j of this segment: wait for the last of their MMAs, then rescale
-          const int gp = gj - 1;
-          if (!mbar_wait(&m->p_empty[gp & 1], (gp >> 1) & 1, a.err)) {
-            m->abort_flag = 1;
-            dead = true;
-            break;
-          }
-          tc_fence_after();
+        if (__any_sync(0xffffffffu, resc) && !dead) {  // rescale O_q: no MMA writes it now
           const float f = resc ? exp2f(m_ref - m_new) : 1.f;
 #pragma unroll
           for (int c = 0; c < 128 / 16; ++c) {
             float o[16];
-            tmem_ld16(tbase + lane_base + 256 + c * 16, o);
+            tmem_ld16(tO + lb + c * 16, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) o[e] *= f;
-            tmem_st16(tbase + lane_base + 256 + c * 16, o);
+            tmem_st16(tO + lb + c * 16, o);
           }
           tmem_wait_st();
-          if (resc) {
-            l_sum *= f;
-            m_ref = m_new;
-          }
+        }
+        if (resc) {
+          l_sum *= exp2f(m_ref - m_new);
+          m_ref = m_new;
         }
         if (m_ref == -INFINITY) m_ref = m_new;  // first visible tile (stays -inf if none)
-        // P_j = 2^(scale * v - m_ref) into shared memory (bf16, K-major, 128-byte swizzle)
-        if (gj >= 2 && !mbar_wait(&m->p_empty[b], ((gj >> 1) & 1) ^ 1, a.err)) {
-          m->abort_flag = 1;
-          dead = true;
-          break;
-        }
-        uint8_t* pb = sP + b * DT_P_BYTES;
-        // a row with nothing visible yet has every v = -inf and gets p = 2^(-inf) = 0 everywhere
+        // pass 2: P = 2^(scale * s - m_ref) as bf16 pairs over columns 0..63 of the tile's S
+        // (chunk c of 32 positions lands on S columns already read); a row with nothing visible
+        // yet has every s masked to -inf and gets p = 0
         const float nm = m_ref == -INFINITY ? -INFINITY : -m_ref;
-        const float sc2 = a.scale_log2;
         float rsv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) rsv[e] = 0.f;
+        if (!dead) {
 #pragma unroll
-        for (int c = 0; c < DT_POS / 8; ++c) {  // 16-byte chunks of 8 positions
-          uint32_t w[4];
+          for (int c = 0; c < DT_POS / 32; ++c) {
+            float x[16], y[16];
+            tmem_ld16(tS + lb + c * 32, x);
+            tmem_ld16(tS + lb + c * 32 + 16, y);
+            tmem_wait_ld();
+            uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = fast_exp2(fmaf(v[c * 8 + 2 * e], sc2, nm));
-            const float p1 = fast_exp2(fmaf(v[c * 8 + 2 * e + 1], sc2, nm));
-            rsv[2 * e] += p0;
-            rsv[2 * e + 1] += p1;
-            w[e] = pack_bf16(p0, p1);
+            for (int e = 0; e < 16; ++e) {
+              const int p0 = P0 + c * 32 + 2 * e;
+              const float a0 = e < 8 ? x[2 * e] : y[2 * e - 16];
+              const float a1 = e < 8 ? x[2 * e + 1] : y[2 * e - 15];
+              const float e0 = fast_exp2(fmaf((vis || p0 <= t) ? a0 : -INFINITY, a.scale_log2, nm));
+              const float e1 = fast_exp2(fmaf((vis || p0 + 1 <= t) ? a1 : -INFINITY, a.scale_log2, nm));
+              rsv[e & 7] += e0 + e1;
+              w[e] = pack_bf16(e0, e1);
+            }
+            tmem_st16u(tS + lb + c * 16, w);
           }
-          const int hh = c >> 3, ch = c & 7;
-          *reinterpret_cast<uint4*>(pb + hh * DT_HALF + row * 128 + ((ch ^ (row & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          tmem_wait_st();
         }
-        const float rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
-        l_sum += rs;
-        if (P0 + DT_POS - 1 > seg_tmax) {
-          // the segment's last tile: zero the V rows after its last position (row = position)
-          if (!mbar_wait(&m->kv_full[s], (gj / DT_NST) & 1, a.err)) {
-            m->abort_flag = 1;
-            dead = true;
-            break;
-          }
-          if (P0 + row > seg_tmax) {
+        l_sum += ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
+        if (P0 + DT_POS - 1 > seg_tmax && qt == 0) {
+          // the segment's last tile: zero the V rows after its last position (query tile A's
+          // softmax does it; B's PV is issued after A's)
+          waitw(&m->kv_full[s], (gj / DT_NST) & 1);
+          if (!dead && P0 + row > seg_tmax) {
             uint8_t* vr = sKV + s * DT_STAGE + DT_KV_BYTES + (row >> 6) * DT_HALF + (row & 63) * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -362,31 +365,28 @@ __global__ void __launch_bounds__(DT_THREADS, 1)
               *reinterpret_cast<uint4*>(vr + DT_HALF / 2 + c * 16) = make_uint4(0, 0, 0, 0);
             }
           }
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // V for the MMA
         }
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // P (and V) for the MMA
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&m->p_full[b]);
+        if (lane == 0 && !dead) mbar_arrive(&m->p_full[qt]);
       }
-      if (!dead && ntile > 0) {
+      if (ntile > 0) {
         const int gl = gbase + ntile - 1;
-        if (!mbar_wait(&m->p_empty[gl & 1], (gl >> 1) & 1, a.err)) {
-          m->abort_flag = 1;
-        } else {
+        waitw(&m->o_done[qt], gl & 1);
+        if (!dead) {
           tc_fence_after();
           const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
           bf16* dst = act ? a.out + ((long long)(tok0 + tok) * a.Hq + g * G + head) * 128 : nullptr;
 #pragma unroll
           for (int c = 0; c < 128 / 16; ++c) {
             float o[16];
-            tmem_ld16(tbase + lane_base + 256 + c * 16, o);
+            tmem_ld16(tO + lb + c * 16, o);
             tmem_wait_ld();
             if (act) {
               uint32_t w[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[2 * e] * inv, o[2 * e + 1] * inv);
-                w[e] = *reinterpret_cast<const uint32_t*>(&h2);
-              }
+              for (int e = 0; e < 8; ++e) w[e] = pack_bf16(o[2 * e] * inv, o[2 * e + 1] * inv);
               *reinterpret_cast<uint4*>(dst + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
               *reinterpret_cast<uint4*>(dst + c * 16 + 8) = make_uint4(w[4], w[5], w[6], w[7]);
             }
@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1)
       }
     }
     __syncthreads();
-    if (tid < 4) m->done[tid] |= m->inseg[tid];
+    if (tid < 8) m->done[tid] |= m->inseg[tid];
     gbase += ntile;
   }
 
@@ -471,7 +471,8 @@ cudaError_t launch_dense_tc(const Geometry& g, const void* q, const void* k_pool
   }
   cudaError_t e = set_smem_once(dense_tc_kernel, DT_SMEM);
   if (e != cudaSuccess) return e;
-  dense_tc_kernel<<<dim3((g.num_q + a.TQ - 1) / a.TQ, g.Hkv), DT_THREADS, DT_SMEM, s>>>(a, tmQ, tmK, tmV);
+  const int nt = DT_NQ * a.TQ;
+  dense_tc_kernel<<<dim3((g.num_q + nt - 1) / nt, g.Hkv), DT_THREADS, DT_SMEM, s>>>(a, tmQ, tmK, tmV);
   return cudaGetLastError();
 }
 
