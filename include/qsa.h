@@ -88,13 +88,19 @@ typedef struct qsa_config {
   float softmax_scale;  /* <= 0 selects 1/sqrt(head_dim) */
   int32_t score_path;   /* qsa_index_score_topk algorithm, every one exact and equal:
                            0 auto: 3 for <= 128 rows when its plan fits, else 2 for <= 256 rows,
-                             else 1;
-                           1 many rows: at idx_dim 128 the tcgen05 tensor-core kernel, whose
-                             unsettled rows the streaming kernel redoes; else the streaming kernel;
+                             else 1, or 5 at idx_dim 128 when the rows' row tiles and the context
+                             are such that spreading the work over every SM saves less than the
+                             stream-K form's own costs (pure geometry);
+                           1 many rows: at idx_dim 128 the tcgen05 tensor-core kernels in
+                             their stream-K form (every SM takes an equal share of the (row tile,
+                             key tile) work), whose unsettled rows the streaming kernel redoes;
+                             else the streaming kernel;
                            2 materialised scores (any shape);
                            3 split lists for few rows (idx_dim 128; 2 when its plan does not fit);
-                           4 the mma.sync streaming kernel alone.
-                           Paths 1 and 3 at idx_dim 128 (and auto, which resolves to them) load
+                           4 the mma.sync streaming kernel alone;
+                           5 the tcgen05 kernel in its single-launch form, one CTA per 128-row
+                             tile (idx_dim 128; 1 otherwise).
+                           Paths 1, 3 and 5 at idx_dim 128 (and auto, which resolves to them) load
                            operands through tensor maps: when the driver offers no tensor-map
                            encoder, qsa_index_score_topk returns QSA_ERR_UNSUPPORTED rather than
                            switch kernels silently.  The resolution itself depends on the shape

@@ -49,7 +49,7 @@ qsa_status_t make_geometry(const qsa_config_t* cfg, const qsa_batch_t* b, Geomet
     return QSA_ERR_INVALID_ARG;
   if (!pow2_le(cfg->num_q_heads / cfg->num_kv_heads, 16)) return QSA_ERR_UNSUPPORTED;
   if (cfg->topk_blocks < 1 || cfg->topk_blocks > 512) return QSA_ERR_UNSUPPORTED;
-  if (cfg->score_path < 0 || cfg->score_path > 4) return QSA_ERR_INVALID_ARG;
+  if (cfg->score_path < 0 || cfg->score_path > 5) return QSA_ERR_INVALID_ARG;
   if ((long long)b->max_pages_per_seq * 64 > (1LL << 30)) return QSA_ERR_UNSUPPORTED;
   g->Hq = cfg->num_q_heads;
   g->Hkv = cfg->num_kv_heads;

@@ -710,10 +710,12 @@ int resolve_score_path(const Geometry& g, int requested) {
   switch (requested) {
     case 1: case 2: case 4: return requested;
     case 3: return score_dec_plan_ok(g) ? 3 : 2;
+    case 5: return g.Di == 128 ? 5 : 1;
     default: break;
   }
   if (g.num_q <= 128 && score_dec_plan_ok(g)) return 3;
-  return g.num_q <= 256 ? 2 : 1;
+  if (g.num_q <= 256) return 2;
+  return g.Di == 128 && !score_tc_stream_pays(g) ? 5 : 1;
 }
 
 // The fast Di = 128 kernels (tcgen05 prefill, split-list decode) load operands through tensor
@@ -723,14 +725,15 @@ int resolve_score_path(const Geometry& g, int requested) {
 int tmap_encode_fn_available() { return tmap_encode_fn() != nullptr; }
 
 bool score_path_runnable(const Geometry& g, int path) {
-  const bool needs_tma = (path == 1 && g.Di == 128) || path == 3;
+  const bool needs_tma = (path == 1 && g.Di == 128) || path == 3 || path == 5;
   return !needs_tma || tmap_encode_fn() != nullptr;
 }
 
 size_t score_workspace_bytes(const Geometry& g, int path) {
-  if (path == 1 || path == 4) {
+  if (path == 1 || path == 4 || path == 5) {
     size_t n = (size_t)g.num_q * stream_cap(g.topk) * 8;
-    if (path == 1 && g.Di == 128) n = std::max(n, score_tc_workspace_bytes(g));
+    if (path == 1 && g.Di == 128) n = std::max(n, score_tc_workspace_bytes(g, true));
+    if (path == 5) n = std::max(n, score_tc_workspace_bytes(g, false));
     return n;
   }
   if (path == 3) return score_dec_workspace_bytes(g);
@@ -738,8 +741,8 @@ size_t score_workspace_bytes(const Geometry& g, int path) {
 }
 
 bool score_redo_offset(const Geometry& g, int path, size_t* off) {
-  if (path == 1 && g.Di == 128) {
-    *off = score_tc_redo_offset(g);
+  if ((path == 1 && g.Di == 128) || path == 5) {
+    *off = score_tc_redo_offset(g, path == 1);
     return true;
   }
   if (path == 3) {
@@ -755,10 +758,11 @@ cudaError_t launch_score_topk(const Geometry& g, int path, const void* idx_q, co
   (void)ws_bytes;
   if (g.num_q == 0) return cudaSuccess;
   const ScoreArgs a = make_args(g, idx_q, idx_w, kcomp, sel, n_sel, sel_scores);
-  if (path == 1 && g.Di == 128) {
-    // tensor-core kernel first; the rows it flags are recomputed by the exact streaming kernel
+  if ((path == 1 && g.Di == 128) || path == 5) {
+    // tensor-core kernels first (stream-K over every SM, or path 5: one CTA per 128-row tile);
+    // the rows they flag are recomputed by the exact streaming kernel
     int32_t* redo = nullptr;
-    cudaError_t e = launch_score_tc(a, g, ws, &redo, s);
+    cudaError_t e = launch_score_tc(a, g, ws, &redo, path == 1, s);
     if (e != cudaSuccess) return e;
     return run_stream<128>(a, g, ws, s, redo);
   }

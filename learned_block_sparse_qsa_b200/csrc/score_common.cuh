@@ -134,10 +134,12 @@ __device__ __forceinline__ void tma3d(uint32_t dst, const CUtensorMap* m, int x,
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn();
 
 // score_tc.cu: the tcgen05 kernel (Di = 128) used by the streaming path.
-size_t score_tc_workspace_bytes(const Geometry& g);
-size_t score_tc_redo_offset(const Geometry& g);  // byte offset of the redo flags [num_q]
+// stream: the stream-K form (every SM) rather than one CTA per 128-row tile.
+bool score_tc_stream_pays(const Geometry& g);
+size_t score_tc_workspace_bytes(const Geometry& g, bool stream);
+size_t score_tc_redo_offset(const Geometry& g, bool stream);  // byte offset of the redo flags [num_q]
 cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int32_t** redo_out,
-                            cudaStream_t s);
+                            bool stream, cudaStream_t s);
 
 // score_dec.cu: decode-sized batches (split warp lists + exact merge; Di = 128).
 bool score_dec_plan_ok(const Geometry& g);        // the split-list plan fits (any driver)

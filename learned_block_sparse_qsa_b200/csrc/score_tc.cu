@@ -53,6 +53,26 @@ constexpr int TC_A_BYTES = 4 * 2 * TC_ROWS * 128;  // 4 heads x 2 K-halves x 128
 constexpr int TC_B_STAGE = 2 * TC_BLK * 128;       // 2 K-halves x 128 rows x 128 B
 constexpr int TC_B_BYTES = TC_NST * TC_B_STAGE;
 constexpr int TC_CAP = 2048;          // candidate slots per half-row
+constexpr int TC_STREAM_CTAS = 148;   // CTAs of the stream-K launch (one per SM of a B200)
+
+// The three launches of the stream-K form (mode 0 is the single-launch form):
+//   mode 1  sample: per row tile, the sampled threshold of every row (tau), the number of full
+//           tiles of the row tile (tiles), empty selections of invalid rows, cleared redo flags;
+//   mode 2  stream: CTA c takes the full tiles [c W, (c+1) W) of the concatenation of every row
+//           tile's tiles (W = ceil(total / TC_STREAM_CTAS)); the part of row tile r that CTA c
+//           covers is an item, and items are numbered r + c (unique: the CTAs' ranges follow
+//           one another, so a later row tile never meets an earlier CTA); each item keeps, per
+//           row and column half, its keys at or above tau in block order (runs, runcnt);
+//   select  (tc_select_kernel) per row: the item runs of its row tile in CTA order, so that each
+//           column half's list is ascending by block, then the exact select.
+struct TcPlan {
+  int mode;
+  float* tau;             // [num_q]
+  int32_t* tiles;         // [R]
+  int32_t* prefix;        // [R + 1]: exclusive prefix of tiles, the total last
+  int32_t* runcnt;        // [(R + TC_STREAM_CTAS) * 128 * 2]
+  u64* runs;              // [(R + TC_STREAM_CTAS) * 128 * 2 * TC_CAP]
+};
 
 struct TcMisc {
   // tfull/tempty[0]: TMEM pair X (heads 0, 1); [1]: pair Y (heads 2, 3)
@@ -67,6 +87,7 @@ struct TcMisc {
   int lim[TC_ROWS];
   int cnt[2][TC_ROWS];
   float thr[2][TC_ROWS];
+  int tiles_acc;  // mode 1: full tiles of the row tile's segments
 };
 // operands + bookkeeping; the dynamic shared-memory base must be 1024-byte aligned (checked)
 constexpr int TC_SMEM = TC_A_BYTES + TC_B_BYTES + (int)((sizeof(TcMisc) + 127) / 128 * 128);
@@ -277,16 +298,17 @@ __device__ __forceinline__ void tc_write_merged(const u64* A, int na, const u64*
 __global__ void __launch_bounds__(TC_THREADS, 1)
     score_tc_kernel(ScoreArgs a, const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB, u64* __restrict__ cand,
-                    int32_t* __restrict__ redo) {
+                    int32_t* __restrict__ redo, TcPlan p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sA = smem;
   uint8_t* sB = smem + TC_A_BYTES;
   TcMisc* m = reinterpret_cast<TcMisc*>(sB + TC_B_BYTES);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row0 = blockIdx.x * TC_ROWS;
+  const int mode = p.mode;
 
   if (smem_addr(smem) & 1023) {  // operand tiles need 1024-byte alignment: leave the rows to the
-    if (tid < TC_ROWS && row0 + tid < a.num_q) redo[row0 + tid] = 1;  // exact streaming kernel
+    if (mode != 2 && tid < TC_ROWS && blockIdx.x * TC_ROWS + tid < a.num_q)  // exact streaming kernel
+      redo[blockIdx.x * TC_ROWS + tid] = 1;
     if (tid == 0) flag_error(a.err, QSA_DEVERR_INTERNAL);
     return;
   }
@@ -312,31 +334,68 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         smem_addr(&m->tmem_base)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
   }
-  if (tid < TC_ROWS) {
-    const int r = row0 + tid;
-    int seq = -1, lim = -1;
-    if (r < a.num_q) {
-      lim = row_limit(a, r, &seq);
-      redo[r] = 0;
-    }
-    m->lim[tid] = lim;
-    const unsigned bal = __ballot_sync(0xffffffffu, lim < 0);  // invalid rows count as done
-    if (lane == 0) m->done[tid >> 5] = bal;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = m->tmem_base;
-  if (warp >= 2) {  // rows that failed validation get an empty selection
-    for (int r = (warp - 2) * 16; r < (warp - 2) * 16 + 16; ++r)
-      if (row0 + r < a.num_q && m->lim[r] < 0)
-        write_empty_selection(row0 + r, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
+
+  // row tiles of this CTA: its own (modes 0, 1), or those its stream range meets (mode 2)
+  int rt_begin = blockIdx.x, rt_end = blockIdx.x + 1;
+  int g_lo = 0, g_hi = 0;  // mode 2: this CTA's range of full tiles
+  if (mode == 2) {
+    const int R = (a.num_q + TC_ROWS - 1) / TC_ROWS;
+    const int total = p.prefix[R];
+    const int W = (total + TC_STREAM_CTAS - 1) / TC_STREAM_CTAS;
+    g_lo = min(blockIdx.x * W, total);
+    g_hi = min(g_lo + W, total);
+    rt_begin = rt_end = 0;
+    if (g_lo < g_hi) {  // first row tile whose range ends after g_lo, last that starts before g_hi
+      int lo = 0, hi = R;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (p.prefix[mid + 1] <= g_lo) lo = mid + 1;
+        else hi = mid;
+      }
+      rt_begin = lo;
+      rt_end = lo;
+      while (rt_end < R && p.prefix[rt_end] < g_hi) ++rt_end;
+    }
   }
 
   uint32_t stage_phase = 0;  // epilogue warps: phase of this warp's staging barrier
   bool stage_dead = false;   // a staging copy never landed: the warp's remaining rows go to redo
   int it_base = 0;  // tiles of earlier segments (all roles count the same tiles)
   int segi = 0;     // segments started (phase of the query-tile barrier)
+  for (int rt = rt_begin; rt < rt_end; ++rt) {
+  const int row0 = rt * TC_ROWS;
+  // mode 2: the part of this row tile's tiles that the CTA covers, and its item slot
+  const int r_lo = mode == 2 ? max(g_lo, p.prefix[rt]) - p.prefix[rt] : 0;
+  const int r_hi = mode == 2 ? min(g_hi, p.prefix[rt + 1]) - p.prefix[rt] : 0;
+  const int slot = rt + blockIdx.x;
+  __syncthreads();  // the previous row tile's state is no longer read
+  if (tid < TC_ROWS) {
+    const int r = row0 + tid;
+    int seq = -1, lim = -1;
+    if (r < a.num_q) {
+      lim = row_limit(a, r, &seq);
+      if (mode != 2) redo[r] = 0;
+    }
+    m->lim[tid] = lim;
+    const unsigned bal = __ballot_sync(0xffffffffu, lim < 0);  // invalid rows count as done
+    if (lane == 0) m->done[tid >> 5] = bal;
+    if (tid == 0) m->tiles_acc = 0;
+  }
+  if (mode == 2 && warp >= 2) {  // every row's run of this item starts empty
+    const int rr = (warp & 3) * 32 + lane, hh = (warp - 2) >> 2;
+    p.runcnt[((long long)slot * TC_ROWS + rr) * 2 + hh] = 0;
+  }
+  __syncthreads();
+  if (mode != 2 && warp >= 2) {  // rows that failed validation get an empty selection
+    for (int r = (warp - 2) * 16; r < (warp - 2) * 16 + 16; ++r)
+      if (row0 + r < a.num_q && m->lim[r] < 0)
+        write_empty_selection(row0 + r, a.sel, a.n_sel, a.sel_scores, a.sel_stride);
+  }
+  int seg_off = 0;  // mode 2: this row tile's tiles before the current segment
   for (;;) {
     __syncthreads();
     if (warp == 0) {  // next segment: the sequence of the first row not yet done
@@ -361,8 +420,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int seg = m->seg;
     if (seg < 0 || m->abort_flag) break;
     const int ntile = (m->nb + TC_BLK - 1) / TC_BLK;
-    const int nsamp = (ntile + TC_SAMPLE - 1) / TC_SAMPLE;
-    const int L = ntile > 0 ? nsamp + ntile : 0;
+    // tiles of this segment in this launch: sample tiles, then full tiles [t_lo, t_hi)
+    int nsamp = (ntile + TC_SAMPLE - 1) / TC_SAMPLE, t_lo = 0, t_hi = ntile;
+    if (mode == 1) t_hi = 0;
+    if (mode == 2) {
+      nsamp = 0;
+      t_lo = min(max(r_lo - seg_off, 0), ntile);
+      t_hi = min(max(r_hi - seg_off, 0), ntile);
+    }
+    if (tid == 0) m->tiles_acc += ntile;
+    seg_off += ntile;
+    const int L = ntile > 0 ? nsamp + max(t_hi - t_lo, 0) : 0;
+    if (mode == 2 && L == 0) {  // nothing of this segment here (every role sees the same)
+      __syncthreads();
+      if (tid < 4) m->done[tid] |= m->inseg[tid];
+      continue;
+    }
 
     if (warp == 0) {
       // ---------------------------------------------------------------- TMA producer
@@ -381,7 +454,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         {
           const int i = i0 + lane / TC_PG;
           if (i < L) {
-            const int tile = i < nsamp ? i * TC_SAMPLE : i - nsamp;
+            const int tile = i < nsamp ? i * TC_SAMPLE : t_lo + i - nsamp;
             const int lp = tile * TC_PG + (lane % TC_PG);
             if (lp < a.max_pages) {  // pages past the table hold only masked blocks: page 0
               const int p = pt[lp];
@@ -464,7 +537,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       for (int k = 0; k < TC_KEEP; ++k) top[k] = -INFINITY;
       float mn = -INFINITY, tau = -INFINITY;
       int cnt = 0;
-      u64* mybuf = cand + ((long long)(row0 + row) * 2 + hf) * TC_CAP;
+      u64* mybuf = mode == 2 ? p.runs + (((long long)slot * TC_ROWS + row) * 2 + hf) * TC_CAP
+                             : cand + ((long long)(row0 + row) * 2 + hf) * TC_CAP;
       const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + hf * 64;
       bool dead = false;
       // Scores of this thread's 64 blocks of tile gi: pair X folded into sc[] and released, then
@@ -538,18 +612,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       // -- row threshold: every epilogue warp arrives here once per segment with tiles
-      if (L > 0) {
+      if (mode == 2) {
+        tau = lim >= 0 ? p.tau[row0 + row] : -INFINITY;  // from the sample launch
+      } else if (L > 0) {
         // a row of at most 2 * TC_CAP candidates keeps every key (each half-row holds at most
         // TC_CAP): a sample of one or two tiles would keep too few of them for the exact select
         m->thr[hf][row] = (lim > a.topk && lim > 2 * TC_CAP) ? mn : -INFINITY;
         epi_sync();
         tau = fminf(m->thr[0][row], m->thr[1][row]);
+        if (mode == 1 && hf == 0 && lim >= 0) p.tau[row0 + row] = tau;
       }
       // -- all tiles: append every key with score >= tau (ascending block order per half-row)
       for (int i = nsamp; i < L; ++i) {
         float sc[64];
         if (!load_scores(it_base + i, sc)) continue;
-        const int bbase = (i - nsamp) * TC_BLK + hf * 64;
+        const int bbase = (t_lo + i - nsamp) * TC_BLK + hf * 64;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           const int nvalid = min(32, lim - bbase - half * 32);  // blocks below the causal limit
@@ -567,12 +644,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       m->cnt[hf][row] = cnt;
+      if (mode == 2 && lim >= 0) p.runcnt[((long long)slot * TC_ROWS + row) * 2 + hf] = cnt;
       // the final select reads the candidate buffers with bulk copies (async proxy)
       asm volatile("fence.proxy.async.global;\n" ::: "memory");
     }
     __syncthreads();  // the segment's tiles are all consumed; stage memory is free
 
-    if (warp >= 2 && !m->abort_flag) {
+    if (mode == 0 && warp >= 2 && !m->abort_flag) {
       // ---------------------------------------------------------------- exact final selection
       // Both half-row lists are ascending by block.  Find the need-th largest key of their union,
       // keep the keys >= it from each list in order, and merge the two by block.
@@ -655,6 +733,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     it_base += L;
     ++segi;
   }
+  if (mode == 1 && tid == 0) p.tiles[rt] = m->tiles_acc;
+  }  // row tiles
 
   // ---------------------------------------------------------------- teardown
   __syncthreads();
@@ -674,6 +754,110 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 }
 
+// Exclusive prefix of the row tiles' tile counts (one warp), the total last.
+__global__ void tc_scan_kernel(const int32_t* __restrict__ tiles, int R, int32_t* __restrict__ prefix) {
+  const int lane = threadIdx.x & 31;
+  int carry = 0;
+  for (int base = 0; base < R; base += 32) {
+    const int v = base + lane < R ? tiles[base + lane] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (base + lane < R) prefix[base + lane] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) prefix[R] = carry;
+}
+
+// The exact final select of the stream-K form, one warp per row: the runs its row tile's items
+// left for the row, in CTA order (so that each column half's list is ascending by block, with a
+// zero key after each odd-length run, below every real key), staged by bulk copies; then the
+// need-th largest key, the keys at or above it kept in place, and a merge by block.
+constexpr int TS_WARPS = 6;
+constexpr int TS_KEYS = 2 * TC_CAP + 2 * (TC_STREAM_CTAS + 1);  // both halves, odd runs padded
+constexpr int TS_REGION = TC_SEL_HIST * 4 + TS_KEYS * 8;
+constexpr int TS_SMEM = TS_WARPS * TS_REGION;
+static_assert(TS_REGION % 16 == 0 && TS_SMEM <= 232448, "select shared memory");
+
+__global__ void __launch_bounds__(TS_WARPS * 32) tc_select_kernel(ScoreArgs a, TcPlan p,
+                                                                 int32_t* __restrict__ redo) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint64_t bar[TS_WARPS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < TS_WARPS) mbar_init(&bar[threadIdx.x], 1);
+  mbar_fence_init();
+  __syncthreads();
+  const int row = blockIdx.x * TS_WARPS + warp;
+  if (row >= a.num_q) return;
+  int seq = -1;
+  const int lim = row_limit(a, row, &seq);
+  if (lim < 0) return;  // the sample launch wrote its empty selection
+  uint8_t* region = smem + warp * TS_REGION;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(region);
+  u64* sk = reinterpret_cast<u64*>(region + TC_SEL_HIST * 4);
+  const int need = min(a.topk, lim);
+  if (need == 0) {
+    tc_write_merged(sk, 0, sk, 0, row, lim, a);
+    return;
+  }
+  const int R = (a.num_q + TC_ROWS - 1) / TC_ROWS;
+  const int rt = row / TC_ROWS, rl = row % TC_ROWS;
+  const int total = p.prefix[R];
+  const int W = (total + TC_STREAM_CTAS - 1) / TC_STREAM_CTAS;
+  const int S = p.prefix[rt], T = p.prefix[rt + 1] - S;
+  if (T <= 0 || W <= 0) {  // no tile of this row was streamed: leave it to the exact kernel
+    if (lane == 0) redo[row] = 1;
+    return;
+  }
+  const int c0 = S / W, c1 = (S + T - 1) / W;
+  int n[2] = {0, 0}, st[2] = {0, 0};  // keys and staged slots (odd runs padded) per half
+  for (int c = c0; c <= c1; ++c)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int k = p.runcnt[((long long)(rt + c) * TC_ROWS + rl) * 2 + h];
+      n[h] += k;
+      st[h] += (min(k, TC_CAP) + 1) & ~1;
+    }
+  if (n[0] > TC_CAP || n[1] > TC_CAP || n[0] + n[1] < need) {
+    if (lane == 0) redo[row] = 1;
+    return;
+  }
+  if (lane == 0) {
+    mbar_arrive_expect_tx(&bar[warp], (uint32_t)(st[0] + st[1]) * 8u);
+    int off = 0;
+    for (int h = 0; h < 2; ++h)
+      for (int c = c0; c <= c1; ++c) {
+        const long long base = ((long long)(rt + c) * TC_ROWS + rl) * 2 + h;
+        const int kr = (p.runcnt[base] + 1) & ~1;
+        if (kr) bulk_g2s(smem_addr(sk + off), p.runs + base * TC_CAP, (uint32_t)kr * 8u, &bar[warp]);
+        off += kr;
+      }
+  }
+  if (!mbar_wait(&bar[warp], 0, a.err)) {  // (error flagged) wait once more for the copies to land
+    mbar_wait(&bar[warp], 0, a.err);
+    if (lane == 0) redo[row] = 1;
+    return;
+  }
+  if (lane == 0) {  // the slot after an odd run holds a stale key: below every real key now
+    int off = 0;
+    for (int h = 0; h < 2; ++h)
+      for (int c = c0; c <= c1; ++c) {
+        const int k = p.runcnt[((long long)(rt + c) * TC_ROWS + rl) * 2 + h];
+        if (k & 1) sk[off + k] = 0ull;
+        off += (k + 1) & ~1;
+      }
+  }
+  __syncwarp();
+  const u64 kth = tc_kth_largest(sk, st[0] + st[1], need, hist);
+  __syncwarp();
+  const int na = tc_keep_inplace(sk, st[0], kth);
+  const int nb = tc_keep_inplace(sk + st[0], st[1], kth);
+  tc_write_merged(sk, na, sk + st[0], nb, row, lim, a);
+}
+
 }  // namespace
 
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
@@ -688,20 +872,58 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
   return fn;
 }
 
-size_t score_tc_redo_offset(const Geometry& g) { return (size_t)g.num_q * 2 * TC_CAP * 8; }
+namespace {
+// Workspace of the stream-K form: runs | runcnt | tau | tiles | prefix | redo flags.
+struct TcStreamWs {
+  size_t runs, runcnt, tau, tiles, prefix, redo, total;
+};
+TcStreamWs stream_ws_layout(const Geometry& g) {
+  auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+  const size_t R = ((size_t)g.num_q + TC_ROWS - 1) / TC_ROWS;
+  const size_t items = R + TC_STREAM_CTAS;
+  TcStreamWs w;
+  w.runs = 0;
+  w.runcnt = w.runs + r256(items * TC_ROWS * 2 * TC_CAP * 8);
+  w.tau = w.runcnt + r256(items * TC_ROWS * 2 * 4);
+  w.tiles = w.tau + r256((size_t)g.num_q * 4);
+  w.prefix = w.tiles + r256(R * 4);
+  w.redo = w.prefix + r256((R + 1) * 4);
+  w.total = w.redo + r256((size_t)g.num_q * 4);
+  return w;
+}
+}  // namespace
 
-size_t score_tc_workspace_bytes(const Geometry& g) {
-  return score_tc_redo_offset(g) + ((size_t)g.num_q * 4 + 255) / 256 * 256;
+// The stream-K form pays when the work it spreads over every SM saves more than its own costs
+// (the sample and select launches, about 100 tiles' worth of one CTA): R row tiles of at most T
+// key tiles take ceil(R / CTAs) * T tile times in the single-launch form, R * T / CTAs + 100 here.
+// Pure geometry: T from the largest position.
+bool score_tc_stream_pays(const Geometry& g) {
+  const long long R = ((long long)g.num_q + TC_ROWS - 1) / TC_ROWS;
+  const long long T = ((long long)g.max_pos / 4 + TC_BLK - 1) / TC_BLK + 1;
+  const long long waves = (R + TC_STREAM_CTAS - 1) / TC_STREAM_CTAS;
+  return R * T / TC_STREAM_CTAS + 100 < waves * T;
 }
 
-// Launch the tensor-core kernel; rows it could not settle are flagged in `redo` (a workspace
-// slice) for the exact streaming kernel, which the caller launches next.
+size_t score_tc_redo_offset(const Geometry& g, bool stream) {
+  return stream ? stream_ws_layout(g).redo : (size_t)g.num_q * 2 * TC_CAP * 8;
+}
+
+size_t score_tc_workspace_bytes(const Geometry& g, bool stream) {
+  if (stream) return stream_ws_layout(g).total;
+  return score_tc_redo_offset(g, false) + ((size_t)g.num_q * 4 + 255) / 256 * 256;
+}
+
+// Launch the tensor-core kernel(s): the single-launch form (one CTA per 128-row tile) or the
+// stream-K form (sample, scan, stream over every SM, select).  Rows they could not settle are
+// flagged in `redo` (a workspace slice) for the exact streaming kernel, which the caller
+// launches next.
 cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int32_t** redo_out,
-                            cudaStream_t s) {
+                            bool stream, cudaStream_t s) {
   auto enc = tmap_encode_fn();
   if (!enc) return cudaErrorNotSupported;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
   u64* cand = static_cast<u64*>(ws);
-  int32_t* redo = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + score_tc_redo_offset(g));
+  int32_t* redo = reinterpret_cast<int32_t*>(wb + score_tc_redo_offset(g, stream));
   *redo_out = redo;
   CUtensorMap tmA, tmB;
   {
@@ -726,8 +948,29 @@ cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int
   }
   cudaError_t e = set_smem_once(score_tc_kernel, TC_SMEM);
   if (e != cudaSuccess) return e;
-  const int tiles = (g.num_q + TC_ROWS - 1) / TC_ROWS;
-  score_tc_kernel<<<tiles, TC_THREADS, TC_SMEM, s>>>(a, tmA, tmB, cand, redo);
+  const int R = (g.num_q + TC_ROWS - 1) / TC_ROWS;
+  TcPlan p{};
+  if (!stream) {
+    p.mode = 0;
+    score_tc_kernel<<<R, TC_THREADS, TC_SMEM, s>>>(a, tmA, tmB, cand, redo, p);
+    return cudaGetLastError();
+  }
+  const TcStreamWs w = stream_ws_layout(g);
+  p.runs = reinterpret_cast<u64*>(wb + w.runs);
+  p.runcnt = reinterpret_cast<int32_t*>(wb + w.runcnt);
+  p.tau = reinterpret_cast<float*>(wb + w.tau);
+  p.tiles = reinterpret_cast<int32_t*>(wb + w.tiles);
+  p.prefix = reinterpret_cast<int32_t*>(wb + w.prefix);
+  p.mode = 1;
+  score_tc_kernel<<<R, TC_THREADS, TC_SMEM, s>>>(a, tmA, tmB, cand, redo, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  tc_scan_kernel<<<1, 32, 0, s>>>(p.tiles, R, p.prefix);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  p.mode = 2;
+  score_tc_kernel<<<TC_STREAM_CTAS, TC_THREADS, TC_SMEM, s>>>(a, tmA, tmB, cand, redo, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = set_smem_once(tc_select_kernel, TS_SMEM)) != cudaSuccess) return e;
+  tc_select_kernel<<<(g.num_q + TS_WARPS - 1) / TS_WARPS, TS_WARPS * 32, TS_SMEM, s>>>(a, p, redo);
   return cudaGetLastError();
 }
 

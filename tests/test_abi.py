@@ -64,7 +64,7 @@ def test_workspace_sizes_are_host_computable():
     ("block_tokens", 8, q.QSA_ERR_UNSUPPORTED), ("idx_heads", 2, q.QSA_ERR_UNSUPPORTED),
     ("head_dim", 96, q.QSA_ERR_UNSUPPORTED), ("topk_blocks", 0, q.QSA_ERR_UNSUPPORTED),
     ("topk_blocks", 513, q.QSA_ERR_UNSUPPORTED), ("num_q_heads", 6, q.QSA_ERR_INVALID_ARG),
-    ("page_tokens", 32, q.QSA_ERR_UNSUPPORTED), ("score_path", 5, q.QSA_ERR_INVALID_ARG)])
+    ("page_tokens", 32, q.QSA_ERR_UNSUPPORTED), ("score_path", 6, q.QSA_ERR_INVALID_ARG)])
 def test_invalid_config_rejected_before_launch(field, value, status):
     cfg = q.QsaConfig.make(32, 4, 128, 128)
     setattr(cfg, field, value)
@@ -101,7 +101,7 @@ def test_redo_flags_live_in_the_score_workspace():
     and split-list paths, none for the materialised and plain streaming paths."""
     b = mk_batch(num_q=16384, max_pages=16384, num_pages=16384, max_pos=1048575)
     ws = 1 << 40
-    for path, has in [(1, True), (2, False), (4, False)]:
+    for path, has in [(1, True), (2, False), (4, False), (5, True)]:
         cfg = q.QsaConfig.make(32, 4, 128, 128, score_path=path)
         n = q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK)
         p = q.qsa_index_score_redo_flags(cfg, b, ws, n)

@@ -2,7 +2,10 @@
 branches (rows of at most 4,096 candidates keep every key; longer rows -- every row of a long-
 context chunk -- keep the keys at or above a threshold taken from a sample of tiles), ragged
 multi-sequence row tiles, and the exact fallback for rows the fast kernel cannot settle.  The
-redo flags the score call leaves in its workspace show which kernel produced each checked row."""
+redo flags the score call leaves in its workspace show which kernel produced each checked row.
+Path 1 runs the tensor-core kernels in their stream-K form (every SM takes an equal share of the
+row tiles' key tiles); path 5 runs the single-launch form (one CTA per 128-row tile); the two must
+give identical selections."""
 import numpy as np
 import pytest
 
@@ -49,17 +52,18 @@ def check_rows(run, rows, integer, topk=None, w_bits=None, model=False):
     return settled if model else o
 
 
-def run_positive_weights(c, **kw):
+def run_positive_weights(c, score_path=1, **kw):
     """Integer inputs with head weights in {1, 2, 3} (positive, as in the pages' workloads)."""
-    run = Run(c, integer=True, score_path=1, **kw)
+    run = Run(c, integer=True, score_path=score_path, **kw)
     w = positive_int_weights(host(c, True).idx_w(np.arange(c.num_q)))
     run.di.idx_w.copy_(torch.from_numpy(w.view(np.int16)).view(torch.bfloat16))
     return run.step(), w
 
 
-def test_tc_prefill_integer_exact_all_rows():
+@pytest.mark.parametrize("path", [1, 5], ids=["stream_k", "single_launch"])
+def test_tc_prefill_integer_exact_all_rows(path):
     """Rows of at most 2,048 candidates: the keep-every-key branch, no row handed over."""
-    run = Run(TC_PREFILL, integer=True, score_path=1).step()
+    run = Run(TC_PREFILL, integer=True, score_path=path).step()
     check_rows(run, range(TC_PREFILL.num_q), True)
     assert run.runner.error_bits() == 0
     assert not run.redo_flags().any()
@@ -69,12 +73,13 @@ SAMPLED = Config("tc_sampled_chunk4096_ctx65536", "prefill", 1, 65536, 4096, 8, 
                  shuffle_pages=True, seed=0x7C04)
 
 
-def test_tc_sampled_threshold_integer_exact_all_rows():
+@pytest.mark.parametrize("path", [1, 5], ids=["stream_k", "single_launch"])
+def test_tc_sampled_threshold_integer_exact_all_rows(path):
     """A 4,096-token chunk at 65,536 tokens of context: every row has 15,360-16,383 candidates,
     so every row takes the sampled-threshold branch.  All rows bit-exact against the oracle, and
     each row's redo flag equals the model of the branch, which settles every row here: the
     checked selections are the tensor-core kernel's own."""
-    run, w = run_positive_weights(SAMPLED)
+    run, w = run_positive_weights(SAMPLED, score_path=path)
     settled = check_rows(run, range(SAMPLED.num_q), True, w_bits=w, model=True)
     assert settled == SAMPLED.num_q
     assert run.runner.error_bits() == 0
@@ -94,11 +99,13 @@ KEEP_ALL_EDGE = Config("tc_keepall_chunk4096_ctx16384", "prefill", 1, 16384, 409
                        shuffle_pages=True, seed=0x7C05)
 
 
-def test_tc_keep_all_rows_on_both_sides_of_the_staging_limit():
-    """Rows of 3,072-4,095 candidates keep every key.  The final select stages a row's keys in
-    shared memory when they fit (3,456 keys) and reads them in place otherwise: rows on both
-    sides of that limit, every row bit-exact and settled by the tensor-core kernel."""
-    run, w = run_positive_weights(KEEP_ALL_EDGE)
+@pytest.mark.parametrize("path", [1, 5], ids=["stream_k", "single_launch"])
+def test_tc_keep_all_rows_on_both_sides_of_the_staging_limit(path):
+    """Rows of 3,072-4,095 candidates keep every key.  The single-launch form's final select
+    stages a row's keys in shared memory when they fit (3,456 keys) and reads them in place
+    otherwise; the stream-K form stages every row.  Every row bit-exact and settled by the
+    tensor-core kernels."""
+    run, w = run_positive_weights(KEEP_ALL_EDGE, score_path=path)
     _, q_pos = host(KEEP_ALL_EDGE, True).rows()
     lim = q_pos // 4
     assert (lim <= 3456).any() and (lim > 3456).any()
@@ -132,9 +139,10 @@ def test_tc_prefill_random_sampled_rows_and_attention():
         check_attention(o["out"][r], o["lse"][r], ref_o, ref_lse)
 
 
-def test_tc_two_sequences_in_one_row_tile():
+@pytest.mark.parametrize("path", [1, 5], ids=["stream_k", "single_launch"])
+def test_tc_two_sequences_in_one_row_tile(path):
     c = Config("tc_ragged_b3", "prefill", 3, 4096, 100, 8, 2, 64, 4, 128, shuffle_pages=True, seed=0x7C02)
-    run = Run(c, integer=True, score_path=1).step()
+    run = Run(c, integer=True, score_path=path).step()
     check_rows(run, range(c.num_q), True)
 
 
@@ -182,8 +190,22 @@ def test_tc_fallback_on_decreasing_scores(ctx, n_new):
         assert bool(redo[r]) == (t // 4 > 4096)  # only the sampled branch is defeated
 
 
-def test_tc_decode_shaped_tile_with_four_sequences():
+@pytest.mark.parametrize("path", [1, 5], ids=["stream_k", "single_launch"])
+def test_tc_decode_shaped_tile_with_four_sequences(path):
     """4 sequences x 4 positions share one 128-row tile: four segments processed in turn."""
     c = Config("tc_decode_b4x4", "decode", 4, 8192, 4, 8, 2, 64, 4, 128, shuffle_pages=True, seed=0x7C03)
-    run = Run(c, integer=True, score_path=1).step()
+    run = Run(c, integer=True, score_path=path).step()
     check_rows(run, range(c.num_q), True)
+
+
+def test_tc_stream_k_equals_single_launch_c2_random():
+    """The C2 chunk on random inputs: the stream-K form and the single-launch form select the
+    same blocks with the same scores on every row."""
+    c = CONFIGS["C2"]
+    a = Run(c, integer=False, score_path=1).step()
+    sel1, n1, sc1 = a.sel.cpu(), a.n_sel.cpu(), a.sel_scores.cpu().numpy()
+    r1 = a.redo_flags()
+    b = Run(c, integer=False, score_path=5).step()
+    assert torch.equal(n1, b.n_sel.cpu()) and torch.equal(sel1, b.sel.cpu())
+    assert np.array_equal(np.nan_to_num(sc1, nan=-1.0), np.nan_to_num(b.sel_scores.cpu().numpy(), nan=-1.0))
+    assert not r1.any() and not b.redo_flags().any()
