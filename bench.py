@@ -731,6 +731,8 @@ def main():
     ap.add_argument("--fused", action="store_true", help="with a decode --case: the one-launch step too")
     ap.add_argument("--train", action="store_true",
                     help="with a prefill --case: the attention backward and the distillation signal")
+    ap.add_argument("--dense", action="store_true",
+                    help="with a --case: the dense paged-GQA baseline on the same inputs too")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -771,6 +773,12 @@ def main():
                 w, max(args.steps, 1), max(args.warmup, 1), lambda: flush_buf.zero_())
         if not decode and args.train:
             res["training_kernels"] = training_kernels_case(w, max(args.steps, 1))
+        if args.dense:
+            d = w.di
+            out = torch.empty_like(w.out)
+            run = lambda: w.runner.dense(w.b, q=d.q, k_pool=d.k_pool, v_pool=d.v_pool, out=out,
+                                         decode=decode)
+            res["dense_ms"] = _time_ms(torch, run, max(args.steps, 1))
         print(json.dumps(res))
         return
 

@@ -778,7 +778,9 @@ __global__ void tc_scan_kernel(const int32_t* __restrict__ tiles, int R, int32_t
 // need-th largest key, the keys at or above it kept in place, and a merge by block.
 constexpr int TS_WARPS = 6;
 constexpr int TS_KEYS = 2 * TC_CAP + 2 * (TC_STREAM_CTAS + 1);  // both halves, odd runs padded
-constexpr int TS_REGION = TC_SEL_HIST * 4 + TS_KEYS * 8;
+constexpr int TS_RUNS = 2 * (TC_STREAM_CTAS + 1);                // runs of one row, at most
+constexpr int TS_TABLE = (TS_RUNS * 8 + 15) / 16 * 16;           // (count, offset) per run
+constexpr int TS_REGION = TC_SEL_HIST * 4 + TS_TABLE + TS_KEYS * 8;
 constexpr int TS_SMEM = TS_WARPS * TS_REGION;
 static_assert(TS_REGION % 16 == 0 && TS_SMEM <= 232448, "select shared memory");
 
@@ -797,7 +799,8 @@ __global__ void __launch_bounds__(TS_WARPS * 32) tc_select_kernel(ScoreArgs a, T
   if (lim < 0) return;  // the sample launch wrote its empty selection
   uint8_t* region = smem + warp * TS_REGION;
   uint32_t* hist = reinterpret_cast<uint32_t*>(region);
-  u64* sk = reinterpret_cast<u64*>(region + TC_SEL_HIST * 4);
+  int* table = reinterpret_cast<int*>(region + TC_SEL_HIST * 4);
+  u64* sk = reinterpret_cast<u64*>(region + TC_SEL_HIST * 4 + TS_TABLE);
   const int need = min(a.topk, lim);
   if (need == 0) {
     tc_write_merged(sk, 0, sk, 0, row, lim, a);
@@ -813,42 +816,61 @@ __global__ void __launch_bounds__(TS_WARPS * 32) tc_select_kernel(ScoreArgs a, T
     return;
   }
   const int c0 = S / W, c1 = (S + T - 1) / W;
-  int n[2] = {0, 0}, st[2] = {0, 0};  // keys and staged slots (odd runs padded) per half
-  for (int c = c0; c <= c1; ++c)
+  const int nr = 2 * (c1 - c0 + 1);  // runs: half-major, then CTA order
+  // every lane reads the counts of its runs at once; the staged slots follow by a warp scan
+  int n[2] = {0, 0}, st[2] = {0, 0};
+  for (int b0 = 0; b0 < nr; b0 += 32) {
+    const int i = b0 + lane;
+    const int h = i / (c1 - c0 + 1), c = c0 + i % (c1 - c0 + 1);
+    const int k = i < nr ? p.runcnt[((long long)(rt + c) * TC_ROWS + rl) * 2 + h] : 0;
+    const int kr = (min(k, TC_CAP) + 1) & ~1;
+    int incl = kr;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int k = p.runcnt[((long long)(rt + c) * TC_ROWS + rl) * 2 + h];
-      n[h] += k;
-      st[h] += (min(k, TC_CAP) + 1) & ~1;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
     }
-  if (n[0] > TC_CAP || n[1] > TC_CAP || n[0] + n[1] < need) {
+    if (i < nr) {
+      // staging offset of this run: the slots of every earlier run (earlier chunks included)
+      const int off = st[0] + st[1] + incl - kr;
+      table[2 * i] = k;  // (count, offset) of run i, for the copies and the pads below
+      table[2 * i + 1] = off;
+    }
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const bool mine = i < nr && h == h2;
+      int kk = mine ? k : 0, ss = mine ? kr : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        kk += __shfl_xor_sync(0xffffffffu, kk, o);
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      }
+      n[h2] += kk;
+      st[h2] += ss;
+    }
+  }
+  __syncwarp();
+  if (n[0] > TC_CAP || n[1] > TC_CAP || n[0] + n[1] < need || nr > TS_RUNS) {
     if (lane == 0) redo[row] = 1;
     return;
   }
-  if (lane == 0) {
-    mbar_arrive_expect_tx(&bar[warp], (uint32_t)(st[0] + st[1]) * 8u);
-    int off = 0;
-    for (int h = 0; h < 2; ++h)
-      for (int c = c0; c <= c1; ++c) {
-        const long long base = ((long long)(rt + c) * TC_ROWS + rl) * 2 + h;
-        const int kr = (p.runcnt[base] + 1) & ~1;
-        if (kr) bulk_g2s(smem_addr(sk + off), p.runs + base * TC_CAP, (uint32_t)kr * 8u, &bar[warp]);
-        off += kr;
-      }
+  if (lane == 0) mbar_arrive_expect_tx(&bar[warp], (uint32_t)(st[0] + st[1]) * 8u);
+  __syncwarp();
+  for (int i = lane; i < nr; i += 32) {  // one lane per run issues its copy
+    const int h = i / (c1 - c0 + 1), c = c0 + i % (c1 - c0 + 1);
+    const int k = table[2 * i], off = table[2 * i + 1];
+    const int kr = (k + 1) & ~1;
+    const long long base = ((long long)(rt + c) * TC_ROWS + rl) * 2 + h;
+    if (kr) bulk_g2s(smem_addr(sk + off), p.runs + base * TC_CAP, (uint32_t)kr * 8u, &bar[warp]);
   }
   if (!mbar_wait(&bar[warp], 0, a.err)) {  // (error flagged) wait once more for the copies to land
     mbar_wait(&bar[warp], 0, a.err);
     if (lane == 0) redo[row] = 1;
     return;
   }
-  if (lane == 0) {  // the slot after an odd run holds a stale key: below every real key now
-    int off = 0;
-    for (int h = 0; h < 2; ++h)
-      for (int c = c0; c <= c1; ++c) {
-        const int k = p.runcnt[((long long)(rt + c) * TC_ROWS + rl) * 2 + h];
-        if (k & 1) sk[off + k] = 0ull;
-        off += (k + 1) & ~1;
-      }
+  for (int i = lane; i < nr; i += 32) {  // the slot after an odd run holds a stale key: below
+    const int k = table[2 * i];  // every real key now
+    if (k & 1) sk[table[2 * i + 1] + k] = 0ull;
   }
   __syncwarp();
   const u64 kth = tc_kth_largest(sk, st[0] + st[1], need, hist);
