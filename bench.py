@@ -648,6 +648,16 @@ def _time_ms(torch, fn, reps: int) -> float:
     return statistics.mean(a.elapsed_time(b) for a, b in ev)
 
 
+def _distill_workspace(cfg, b, device):
+    """Workspace of the distillation call (None and 0 where its form needs none)."""
+    import torch
+
+    from learned_block_sparse_qsa_b200 import QSA_OP_DISTILL_KL, qsa_workspace_size
+
+    n = qsa_workspace_size(cfg, b, QSA_OP_DISTILL_KL)
+    return (torch.empty(n, dtype=torch.uint8, device=device) if n else None), n
+
+
 def training_kernels(w: Workload, peaks, reps: int = 3):
     """The training-side kernels on the prefill workload's device inputs: the sparse attention
     backward (16,384 rows at 1M context, gradients accumulated into fp32 cache-shaped pools), and
@@ -680,8 +690,10 @@ def training_kernels(w: Workload, peaks, reps: int = 3):
     kl = torch.empty(cd.num_q, dtype=torch.float32, device=d.q.device)
     dd = wd.di
     wd.step(False)  # compresses the chunk's keys
+    dws, dn = _distill_workspace(wd.cfg, wd.b, d.q.device)
     dist_ms = _time_ms(torch, lambda: qsa_index_distill_kl(
-        wd.cfg, wd.b, dd.q, dd.k_pool, dd.idx_q, dd.idx_w, dd.kcomp_pool, kl), reps)
+        wd.cfg, wd.b, dd.q, dd.k_pool, dd.idx_q, dd.idx_w, dd.kcomp_pool, kl, workspace=dws,
+        ws_bytes=dn), reps)
     t = np.asarray(wd.q_pos_host, dtype=np.int64)
     dist_flops = int((2 * cd.Hq * cd.D * (t + 1 + 4 * (t // 4))).sum() + (2 * 4 * cd.Di * (t // 4)).sum())
     del wd
@@ -693,7 +705,7 @@ def training_kernels(w: Workload, peaks, reps: int = 3):
                                  "note": "dk/dv added to fp32 pools by vector atomics"},
         "distill_kl": {"workload": cd.name, "ms": dist_ms, "tflops": dist_flops / (dist_ms * 1e-3) / 1e12,
                        "peak_tflops": peaks["tf"], "frac": dist_flops / (dist_ms * 1e-3) / 1e12 / peaks["tf"],
-                       "kernel": "mma.sync"},
+                       "kernel": "tcgen05" if dn else "mma.sync"},
     }
 
 
@@ -713,8 +725,10 @@ def training_kernels_case(w: Workload, reps: int):
     kl = torch.empty(c.num_q, dtype=torch.float32, device=d.q.device)
     bwd = _time_ms(torch, lambda: qsa_sparse_attn_backward(w.cfg, b, d.q, d.k_pool, d.v_pool, w.sel, w.n_sel,
                                                            w.out, lse, dout, dq, dk, dv), reps)
+    dws, dn = _distill_workspace(w.cfg, b, d.q.device)
     dst = _time_ms(torch, lambda: qsa_index_distill_kl(w.cfg, b, d.q, d.k_pool, d.idx_q, d.idx_w,
-                                                       d.kcomp_pool, kl), reps)
+                                                       d.kcomp_pool, kl, workspace=dws,
+                                                       ws_bytes=dn), reps)
     return {"sparse_attn_backward_ms": bwd, "distill_kl_ms": dst}
 
 

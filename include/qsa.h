@@ -73,7 +73,8 @@ typedef enum qsa_op {
   QSA_OP_SPARSE_ATTN_DECODE = 2,
   QSA_OP_DENSE_ATTN_DECODE = 3,
   QSA_OP_MERGE_CANDIDATES = 4, /* num_splits = number of parts */
-  QSA_OP_DECODE_STEP = 5       /* num_splits as passed to qsa_decode_step */
+  QSA_OP_DECODE_STEP = 5,      /* num_splits as passed to qsa_decode_step */
+  QSA_OP_DISTILL_KL = 6        /* qsa_index_distill_kl; num_splits unused */
 } qsa_op_t;
 
 typedef struct qsa_config {
@@ -307,11 +308,16 @@ qsa_status_t qsa_sparse_attn_backward(const qsa_config_t* cfg, const qsa_batch_t
  * Optional outputs: lse (float [num_q, Hq], natural-log normaliser of each head's dense softmax)
  * and teacher (float [num_q, ld], ld >= max_pos/4: the teacher distribution, entries b >= t/4
  * untouched).  Needs keys of positions 0..t in k_pool and the compressed keys of blocks < t/4;
- * reads no values.  No workspace.  A dense computation (two passes of q.k over the context). */
+ * reads no values.  A dense computation (two passes of q.k over the context).  At head_dim 128
+ * with 8 query heads per KV head it runs on the tensor cores and needs a workspace of
+ * qsa_workspace_size(..., QSA_OP_DISTILL_KL, 0, ...) bytes (block masses and indexer scores of
+ * every row: 8 * num_q * (max_pos/4 + 1) bytes, rounded; QSA_ERR_WORKSPACE if smaller;
+ * QSA_ERR_UNSUPPORTED when the driver has no tensor-map encoder); other shapes need none. */
 qsa_status_t qsa_index_distill_kl(const qsa_config_t* cfg, const qsa_batch_t* batch,
                                   const void* q, const void* k_pool, const void* idx_q,
                                   const void* idx_w, const void* kcomp_pool, float* kl, float* lse,
-                                  float* teacher, int64_t ld, qsa_stream_t stream);
+                                  float* teacher, int64_t ld, void* workspace, size_t ws_bytes,
+                                  qsa_stream_t stream);
 
 /* No counterpart in the article: a self-test of failure detection.  Every pipelined kernel waits
  * on mbarriers with a bounded wait that, when it runs out, sets QSA_DEVERR_TIMEOUT in *err_flag

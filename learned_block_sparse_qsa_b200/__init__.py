@@ -24,7 +24,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA = 0, 1, 2, 3, 4
 QSA_OP_INDEX_SCORE_TOPK, QSA_OP_SPARSE_ATTN_DECODE, QSA_OP_DENSE_ATTN_DECODE = 1, 2, 3
-QSA_OP_MERGE_CANDIDATES, QSA_OP_DECODE_STEP = 4, 5
+QSA_OP_MERGE_CANDIDATES, QSA_OP_DECODE_STEP, QSA_OP_DISTILL_KL = 4, 5, 6
 DEVERR = {"SEQ": 1, "POS": 2, "PAGE": 4, "GROUP": 8, "SEL": 16, "TIMEOUT": 32, "INTERNAL": 64}
 
 
@@ -103,7 +103,8 @@ _SIGS = {
                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                            c_void_p, c_void_p]),
     "qsa_index_distill_kl": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
-                                       c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
+                                       c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_size_t,
+                                       c_void_p]),
     "qsa_dense_attn_prefill": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_void_p]),
     "qsa_dense_attn_decode": (c_int32, [_S, _B, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -239,11 +240,12 @@ def qsa_sparse_attn_backward(cfg, batch, q, k_pool, v_pool, sel, n_sel, out, lse
 
 
 def qsa_index_distill_kl(cfg, batch, q, k_pool, idx_q, idx_w, kcomp_pool, kl, lse=None,
-                         teacher=None, ld=0, stream=None):
+                         teacher=None, ld=0, workspace=None, ws_bytes=0, stream=None):
     """Per-row KL(block-pooled dense attention || indexer softmax); see include/qsa.h."""
     _check(_lib.qsa_index_distill_kl(ctypes.byref(cfg), ctypes.byref(batch), _p(q), _p(k_pool),
                                      _p(idx_q), _p(idx_w), _p(kcomp_pool), _p(kl), _p(lse),
-                                     _p(teacher), int(ld), _stream(stream)),
+                                     _p(teacher), int(ld), _p(workspace), int(ws_bytes),
+                                     _stream(stream)),
            "qsa_index_distill_kl")
 
 

@@ -117,6 +117,9 @@ qsa_status_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_batch_t* batc
       *bytes = s > 1 ? qsa::dense_decode_workspace_bytes(g, s) : 0;
       return QSA_OK;
     }
+    case QSA_OP_DISTILL_KL:
+      *bytes = qsa::distill_tc_shape(g) ? qsa::distill_tc_workspace_bytes(g) : 0;
+      return QSA_OK;
   }
   return QSA_ERR_INVALID_ARG;
 }
@@ -320,7 +323,8 @@ qsa_status_t qsa_sparse_attn_backward(const qsa_config_t* cfg, const qsa_batch_t
 qsa_status_t qsa_index_distill_kl(const qsa_config_t* cfg, const qsa_batch_t* batch,
                                   const void* q, const void* k_pool, const void* idx_q,
                                   const void* idx_w, const void* kcomp_pool, float* kl, float* lse,
-                                  float* teacher, int64_t ld, qsa_stream_t stream) {
+                                  float* teacher, int64_t ld, void* workspace, size_t ws_bytes,
+                                  qsa_stream_t stream) {
   Geometry g;
   qsa_status_t st = make_geometry(cfg, batch, &g, true);
   if (st != QSA_OK || g.num_q == 0) return st;
@@ -329,6 +333,14 @@ qsa_status_t qsa_index_distill_kl(const qsa_config_t* cfg, const qsa_batch_t* ba
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k_pool) |
        reinterpret_cast<uintptr_t>(idx_q) | reinterpret_cast<uintptr_t>(kcomp_pool)) & 15)
     return QSA_ERR_INVALID_ARG;
+  if (qsa::distill_tc_shape(g)) {  // the tensor-core form
+    if (!qsa::tmap_encode_fn_available()) return QSA_ERR_UNSUPPORTED;
+    if (!workspace || ws_bytes < qsa::distill_tc_workspace_bytes(g) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 15))
+      return QSA_ERR_WORKSPACE;
+    return from_cuda(qsa::launch_distill_tc(g, q, k_pool, idx_q, idx_w, kcomp_pool, kl, lse, teacher,
+                                            ld, workspace, (cudaStream_t)stream));
+  }
   return from_cuda(qsa::launch_distill(g, q, k_pool, idx_q, idx_w, kcomp_pool, kl, lse, teacher,
                                        ld, (cudaStream_t)stream));
 }

@@ -81,6 +81,12 @@ cudaError_t launch_sparse_attn_bwd(const Geometry& g, const void* q, const void*
                                    float* dk_pool, float* dv_pool, cudaStream_t s);
 
 // distill.cu
+// distill_tc.cu: the tensor-core form (head_dim 128, 8 query heads per KV head)
+bool distill_tc_shape(const Geometry& g);
+size_t distill_tc_workspace_bytes(const Geometry& g);
+cudaError_t launch_distill_tc(const Geometry& g, const void* q, const void* k_pool, const void* idx_q,
+                              const void* idx_w, const void* kcomp, float* kl, float* lse, float* teacher,
+                              int64_t ld, void* ws, cudaStream_t s);
 cudaError_t launch_distill(const Geometry& g, const void* q, const void* k_pool, const void* idx_q,
                            const void* idx_w, const void* kcomp, float* kl, float* lse,
                            float* teacher, int64_t ld, cudaStream_t s);

@@ -23,6 +23,16 @@ KL_ATOL, KL_RTOL = 2e-3, 2e-3
 P_ATOL, P_RTOL = 1e-6, 2e-3
 LSE_ATOL, LSE_RTOL = 1e-3, 1e-4
 
+
+def workspace(run):
+    """The call's workspace (tensor-core form at head_dim 128 with 8 heads per KV head; none
+    otherwise)."""
+    from learned_block_sparse_qsa_b200 import QSA_OP_DISTILL_KL, qsa_workspace_size
+
+    n = qsa_workspace_size(run.cfg, run.b, QSA_OP_DISTILL_KL)
+    return (torch.empty(n, dtype=torch.uint8, device="cuda") if n else None), n
+
+
 CASES = {
     "C1_4q1kv_d64_di32": CONFIGS["C1"],
     "b2_32q4kv_d128_di128": Config("distill_b2", "prefill", 2, 8192, 300, 32, 4, 128, 4, 128,
@@ -45,9 +55,10 @@ def test_distill_kl_matches_oracle(name):
     kl = torch.full((c.num_q,), float("nan"), dtype=torch.float32, device="cuda")
     lse = torch.full((c.num_q, c.Hq), float("nan"), dtype=torch.float32, device="cuda")
     teacher = torch.full((c.num_q, ld), float("nan"), dtype=torch.float32, device="cuda")
+    ws, n = workspace(run)
     run.runner.clear_error()
     qsa_index_distill_kl(run.cfg, run.b, d.q, d.k_pool, d.idx_q, d.idx_w, d.kcomp_pool, kl, lse,
-                         teacher, ld)
+                         teacher, ld, ws, n)
     torch.cuda.synchronize()
     assert run.runner.error_bits() == 0
     g_kl, g_lse, g_p = kl.cpu().numpy(), lse.cpu().numpy(), teacher.cpu().numpy()
@@ -71,16 +82,20 @@ def test_distill_kl_matches_oracle(name):
         assert np.all(np.isnan(g_p[r, n:]))   # entries b >= t/4 untouched
 
 
-def test_distill_invalid_rows_flagged_and_nan():
+@pytest.mark.parametrize("base", ["C1", "d128_g8"])
+def test_distill_invalid_rows_flagged_and_nan(base):
     from learned_block_sparse_qsa_b200 import qsa_index_distill_kl
 
-    c = CONFIGS["C1"].replace(ctx=512, n_new=512)
+    c = (CONFIGS["C1"] if base == "C1" else CASES["b2_32q4kv_d128_di128"]).replace(
+        batch=1, ctx=512, n_new=512, needles=0)
     run = Run(c, integer=False).step()
     d = run.di
     run.di.q_pos[7] = 100000          # beyond the page table
     kl = torch.zeros(c.num_q, dtype=torch.float32, device="cuda")
+    ws, n = workspace(run)
     run.runner.clear_error()
-    qsa_index_distill_kl(run.cfg, run.b, d.q, d.k_pool, d.idx_q, d.idx_w, d.kcomp_pool, kl)
+    qsa_index_distill_kl(run.cfg, run.b, d.q, d.k_pool, d.idx_q, d.idx_w, d.kcomp_pool, kl,
+                         workspace=ws, ws_bytes=n)
     torch.cuda.synchronize()
     assert run.runner.error_bits() & 2
     g = kl.cpu().numpy()
