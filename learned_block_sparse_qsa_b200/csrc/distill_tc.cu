@@ -13,12 +13,14 @@
 // Three launches:
 //   distill_tc_kernel  CTA = two query tiles of 128 rows (16 tokens x the 8 query heads of one KV
 //                      head each) sharing every K tile; two passes over the context with S = Q K^T
-//                      in tensor memory (double-buffered per query tile).  Pass 1: each row's
-//                      running maximum and sum in base 2 (its dense log-sum-exp).  Pass 2: the
-//                      probabilities 2^(scale s - lse), summed within each 4-position block, then
-//                      over the 8 heads of the token by a shuffle reduce-scatter (each lane ends
-//                      with 4 block sums), added into the block masses of the token in global
-//                      memory (one reduction per KV head and block).
+//                      in tensor memory (double-buffered per query tile).  Eight softmax warps per
+//                      query tile: a warp reads 32 rows (its lane quarter) x 64 of the tile's 128
+//                      columns.  Pass 1: each row's running maximum and sum in base 2 per column
+//                      half, combined once through shared memory (the row's dense log-sum-exp).
+//                      Pass 2: the probabilities 2^(scale s - lse), summed within each 4-position
+//                      block, then over the 8 heads of the token by a shuffle reduce-scatter (each
+//                      lane ends with 2 block sums), added into the block masses of the token in
+//                      global memory (one 8-byte reduction per KV head and block pair).
 //   scores             the indexer scores of every candidate (the materialised scoring kernel).
 //   distill_finish     one warp per row: M = sum m, A = sum m ln m, B = sum m s and the
 //                      log-sum-exp of s over the candidates; KL = A/M - ln M - B/M + lse(s); the
@@ -37,7 +39,8 @@ constexpr int DK_G = 8;       // query heads per KV head of this layout
 constexpr int DK_TQ = DK_ROWS / DK_G;
 constexpr int DK_POS = 128;   // positions per K tile (N of S)
 constexpr int DK_NST = 4;     // K stages
-constexpr int DK_SMW = 4;     // softmax warps per query tile
+constexpr int DK_SMW = 8;     // softmax warps per query tile: 4 lane quarters x 2 column halves
+constexpr int DK_COLS = DK_POS / 2;  // S columns per softmax warp
 constexpr int DK_THREADS = (2 + DK_NQ * DK_SMW) * 32;
 constexpr int DK_HALF = DK_ROWS * 128;   // one 64-column (128-byte) half of a 128-row tile
 constexpr int DK_Q_BYTES = 2 * DK_HALF;  // query tile, K-major: [k-half][row][128 B]
@@ -52,6 +55,7 @@ struct DkMisc {
   int seg, tmax, ntile;
   uint32_t done[1];   // tokens already handled (bit per token; 32 tokens per CTA)
   uint32_t inseg[1];  // tokens of the current segment
+  float2 xch[DK_NQ][DK_ROWS][2];  // pass-1 (max, sum) of each row's two column halves
 };
 constexpr int DK_SMEM = DK_NQ * DK_Q_BYTES + DK_NST * DK_K_BYTES + (int)((sizeof(DkMisc) + 127) / 128 * 128);
 static_assert(DK_SMEM <= 232448, "shared memory budget");
@@ -73,6 +77,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Barrier over `n` threads (a multiple of 32) under id `id` (1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
 
 __device__ __forceinline__ bool dk_valid(const DkArgs& a, int r) {
@@ -143,6 +152,7 @@ __global__ void __launch_bounds__(DK_THREADS, 1)
   }
 
   const int qt = warp >= 2 ? (warp - 2) / DK_SMW : 0;
+  const int half = warp >= 2 ? ((warp - 2) % DK_SMW) / 4 : 0;  // the warp's 64 of the tile's columns
   const int row = 32 * (warp & 3) + lane;
   const int tok = qt * DK_TQ + row / DK_G, head = row % DK_G;
 
@@ -238,7 +248,7 @@ __global__ void __launch_bounds__(DK_THREADS, 1)
       float mx = -INFINITY, sum = 0.f, lse2 = -INFINITY;
       bool dead = false;
       for (int i = 0; i < L; ++i) {
-        const int gj = gbase + i, b = gj & 1, j = i % ntile, P0 = j * DK_POS;
+        const int gj = gbase + i, b = gj & 1, j = i % ntile, P0 = j * DK_POS + half * DK_COLS;
         const bool pass2 = i >= ntile;
         if (!dead) {
           const bool okw = mbar_wait(&m->s_full[qt][b], (gj >> 1) & 1, a.err);
@@ -247,13 +257,13 @@ __global__ void __launch_bounds__(DK_THREADS, 1)
             dead = true;
           }
         }
-        float v[DK_POS];
+        float v[DK_COLS];
         if (!dead) {
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < DK_POS / 16; ++c) {
+          for (int c = 0; c < DK_COLS / 16; ++c) {
             float x[16];
-            tmem_ld16(tbase + lb + qt * 256 + b * 128 + c * 16, x);
+            tmem_ld16(tbase + lb + qt * 256 + b * 128 + half * DK_COLS + c * 16, x);
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[c * 16 + e] = x[e];
           }
@@ -261,21 +271,21 @@ __global__ void __launch_bounds__(DK_THREADS, 1)
           tc_fence_before();
         } else {
 #pragma unroll
-          for (int c = 0; c < DK_POS; ++c) v[c] = -INFINITY;
+          for (int c = 0; c < DK_COLS; ++c) v[c] = -INFINITY;
         }
         __syncwarp();
         if (lane == 0 && !dead) mbar_arrive(&m->s_empty[qt][b]);
-        if (P0 + DK_POS - 1 > t) {  // mask positions after t
+        if (P0 + DK_COLS - 1 > t) {  // mask positions after t
 #pragma unroll
-          for (int c = 0; c < DK_POS; ++c) v[c] = P0 + c <= t ? v[c] : -INFINITY;
+          for (int c = 0; c < DK_COLS; ++c) v[c] = P0 + c <= t ? v[c] : -INFINITY;
         }
         if (!pass2) {
-          // pass 1: running maximum and sum of 2^(scale s) in base 2
+          // pass 1: running maximum and sum of 2^(scale s) in base 2 over this half's columns
           float tm[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) tm[e] = v[e];
 #pragma unroll
-          for (int c = 8; c < DK_POS; c += 8)
+          for (int c = 8; c < DK_COLS; c += 8)
 #pragma unroll
             for (int e = 0; e < 8; ++e) tm[e] = fmaxf(tm[e], v[c + e]);
           const float tmx = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
@@ -286,54 +296,59 @@ __global__ void __launch_bounds__(DK_THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) ps[e] = 0.f;
 #pragma unroll
-            for (int c = 0; c < DK_POS; ++c) ps[c & 7] += fast_exp2(fmaf(v[c], a.scale_log2, -mn));
+            for (int c = 0; c < DK_COLS; ++c) ps[c & 7] += fast_exp2(fmaf(v[c], a.scale_log2, -mn));
             const float ts = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             sum = (mx == -INFINITY ? 0.f : sum * fast_exp2(mx - mn)) + ts;
             mx = mn;
           }
-          if (i == ntile - 1) {  // the row's log-sum-exp, base 2 (and natural, when asked for)
-            lse2 = sum > 0.f ? mx + log2f(sum) : -INFINITY;
-            if (act && a.lse)
+          if (i == ntile - 1) {  // both halves: the row's log-sum-exp, base 2
+            m->xch[qt][row][half] = make_float2(mx, sum);
+            named_bar_sync(1 + qt, DK_SMW * 32);
+            const float2 o = m->xch[qt][row][half ^ 1];
+            const float M2 = fmaxf(mx, o.x);
+            const float S2 = (mx == -INFINITY ? 0.f : sum * fast_exp2(mx - M2)) +
+                             (o.x == -INFINITY ? 0.f : o.y * fast_exp2(o.x - M2));
+            lse2 = S2 > 0.f ? M2 + log2f(S2) : -INFINITY;
+            if (act && a.lse && half == 0)  // natural log
               a.lse[(long long)(tok0 + tok) * a.Hq + g * DK_G + head] = lse2 * 0.69314718055994531f;
           }
         } else {
           // pass 2: block masses of this head's probabilities, then the 8 heads' sum
           const float nl = lse2 == -INFINITY ? -INFINITY : -lse2;
-          float bs[32];
+          float bs[DK_COLS / 4];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
+          for (int k = 0; k < DK_COLS / 4; ++k) {
             float s4 = 0.f;
 #pragma unroll
             for (int e = 0; e < 4; ++e) s4 += fast_exp2(fmaf(v[4 * k + e], a.scale_log2, nl));
             bs[k] = s4;
           }
-          // reduce-scatter over the token's 8 lanes: lane bits 2, 1, 0 pick halves of 16, 8, 4
+          // reduce-scatter over the token's 8 lanes: lane bits 2, 1, 0 pick halves of 8, 4, 2
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
+          for (int k = 0; k < 8; ++k) {
             const bool up = lane & 4;
-            const float keep = up ? bs[16 + k] : bs[k], give = up ? bs[k] : bs[16 + k];
+            const float keep = up ? bs[8 + k] : bs[k], give = up ? bs[k] : bs[8 + k];
             bs[k] = keep + __shfl_xor_sync(0xffffffffu, give, 4);
           }
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
+          for (int k = 0; k < 4; ++k) {
             const bool up = lane & 2;
-            const float keep = up ? bs[8 + k] : bs[k], give = up ? bs[k] : bs[8 + k];
+            const float keep = up ? bs[4 + k] : bs[k], give = up ? bs[k] : bs[4 + k];
             bs[k] = keep + __shfl_xor_sync(0xffffffffu, give, 2);
           }
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 2; ++k) {
             const bool up = lane & 1;
-            const float keep = up ? bs[4 + k] : bs[k], give = up ? bs[k] : bs[4 + k];
+            const float keep = up ? bs[2 + k] : bs[k], give = up ? bs[k] : bs[2 + k];
             bs[k] = keep + __shfl_xor_sync(0xffffffffu, give, 1);
           }
-          const int kb0 = ((lane >> 2) & 1) * 16 + ((lane >> 1) & 1) * 8 + (lane & 1) * 4;
-          if (act && !dead) {
-            float* mrow = a.mass + (long long)(tok0 + tok) * a.ldm;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int blk = P0 / 4 + kb0 + e;
-              if (blk < nb) atomicAdd(mrow + blk, bs[e]);
-            }
+          const int blk = P0 / 4 + ((lane >> 2) & 1) * 8 + ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
+          if (act && !dead && blk < nb) {  // blk is even: the pair is 8-byte aligned
+            float* dst = a.mass + (long long)(tok0 + tok) * a.ldm + blk;
+            if (blk + 1 < nb)
+              atomicAdd(reinterpret_cast<float2*>(dst), make_float2(bs[0], bs[1]));
+            else
+              atomicAdd(dst, bs[0]);
           }
         }
       }
@@ -361,7 +376,9 @@ __global__ void __launch_bounds__(DK_THREADS, 1)
   }
 }
 
-// One warp per row: the KL from the block masses and the indexer scores of its candidates.
+// One warp per row: the KL from the block masses and the indexer scores of its candidates.  Two
+// sweeps of the row: the largest score, then the sums (per-element logarithms and exponentials in
+// fp32, each lane's sums in fp64).
 __global__ void __launch_bounds__(256) distill_finish_kernel(DkArgs a, const float* __restrict__ scores,
                                                             long long lds, float* __restrict__ kl,
                                                             float* __restrict__ teacher, long long ldt) {
@@ -375,34 +392,31 @@ __global__ void __launch_bounds__(256) distill_finish_kernel(DkArgs a, const flo
   const int nb = a.q_pos[r] >> 2;
   const float* mrow = a.mass + (long long)r * a.ldm;
   const float* srow = scores + (long long)r * lds;
-  double M = 0.0, A = 0.0, B = 0.0, smax = -INFINITY, ssum = 0.0;
+  float smax = -INFINITY;
+  for (int b = lane; b < nb; b += 32) smax = fmaxf(smax, srow[b]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+  double M = 0.0, A = 0.0, B = 0.0, Z = 0.0;
   for (int b = lane; b < nb; b += 32) {
-    const double mb = mrow[b], sb = srow[b];
+    const float mb = mrow[b], sb = srow[b];
     M += mb;
-    if (mb > 0.0) A += mb * log(mb);
-    B += mb * sb;
-    if (sb > smax) {
-      ssum = ssum * exp(smax - sb) + 1.0;
-      smax = sb;
-    } else {
-      ssum += exp(sb - smax);
-    }
+    if (mb > 1e-30f) A += (double)(mb * __logf(mb));  // below 1e-30 the term is < 1e-28
+    B += (double)(mb * sb);
+    Z += (double)__expf(sb - smax);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     M += __shfl_xor_sync(0xffffffffu, M, o);
     A += __shfl_xor_sync(0xffffffffu, A, o);
     B += __shfl_xor_sync(0xffffffffu, B, o);
-    const double om = __shfl_xor_sync(0xffffffffu, smax, o), os = __shfl_xor_sync(0xffffffffu, ssum, o);
-    const double nm = om > smax ? om : smax;
-    ssum = (smax == -INFINITY ? 0.0 : ssum * exp(smax - nm)) + (om == -INFINITY ? 0.0 : os * exp(om - nm));
-    smax = nm;
+    Z += __shfl_xor_sync(0xffffffffu, Z, o);
   }
-  if (lane == 0) kl[r] = (nb > 0 && M > 0.0) ? (float)(A / M - log(M) - B / M + smax + log(ssum)) : 0.f;
+  if (lane == 0)
+    kl[r] = (nb > 0 && M > 0.0) ? (float)(A / M - log(M) - B / M + (double)smax + log(Z)) : 0.f;
   if (teacher && nb > 0) {
-    const double inv = M > 0.0 ? 1.0 / M : 0.0;
+    const float inv = M > 0.0 ? (float)(1.0 / M) : 0.f;
     float* trow = teacher + (long long)r * ldt;
-    for (int b = lane; b < nb; b += 32) trow[b] = (float)(mrow[b] * inv);
+    for (int b = lane; b < nb; b += 32) trow[b] = mrow[b] * inv;
   }
 }
 
