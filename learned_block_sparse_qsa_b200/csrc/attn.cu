@@ -53,6 +53,8 @@ struct AttnCfg {
 
 template <int D, int HKV>
 __global__ void __launch_bounds__(AttnCfg<D, HKV>::THREADS, 1) sparse_attn_kernel(AttnArgs a) {
+  chain_wait();
+  chain_release();
   using C = AttnCfg<D, HKV>;
   extern __shared__ __align__(128) uint8_t smem[];
   int* sPos = reinterpret_cast<int*>(smem + C::POS_OFF);
@@ -328,7 +330,18 @@ __global__ void __launch_bounds__(AttnCfg<D, HKV>::THREADS, 1) sparse_attn_kerne
 template <int D, int HKV, int SLC>
 __global__ void __launch_bounds__(SwCfg<D, HKV, SLC>::THREADS, 1) sparse_attn_sw_kernel(AttnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
+  chain_wait();
+  chain_release();
   sparse_attn_sw_body<D, HKV, SLC>(a, blockIdx.x, blockIdx.y, smem);
+}
+
+// Zero n counters, as a chained launch (a memset between two chained kernels would break the
+// chain).  It waits for the previous grid first: that grid may still count on the same words.
+__global__ void zero_u32_kernel(uint32_t* __restrict__ p, int n) {
+  chain_wait();
+  chain_release();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = 0;
 }
 
 // Merge split-K partials: out = sum_s 2^(lse_s - L) o_s, L = log2 sum_s 2^lse_s.
@@ -364,14 +377,13 @@ cudaError_t run_sparse(const AttnArgs& a, int splits, cudaStream_t s) {
     using C = SwCfg<D, HKV, SLC>;
     cudaError_t e = set_smem_once(sparse_attn_sw_kernel<D, HKV, SLC>, C::TOTAL);
     if (e != cudaSuccess) return e;
-    sparse_attn_sw_kernel<D, HKV, SLC><<<dim3(a.num_q, splits), C::THREADS, C::TOTAL, s>>>(a);
-    return cudaGetLastError();
+    return launch_chained(sparse_attn_sw_kernel<D, HKV, SLC>, dim3(a.num_q, splits), dim3(C::THREADS), C::TOTAL, s,
+                          a);
   }
   using C = AttnCfg<D, HKV>;
   cudaError_t e = set_smem_once(sparse_attn_kernel<D, HKV>, C::TOTAL);
   if (e != cudaSuccess) return e;
-  sparse_attn_kernel<D, HKV><<<dim3(a.num_q, splits), C::THREADS, C::TOTAL, s>>>(a);
-  return cudaGetLastError();
+  return launch_chained(sparse_attn_kernel<D, HKV>, dim3(a.num_q, splits), dim3(C::THREADS), C::TOTAL, s, a);
 }
 
 }  // namespace
@@ -440,7 +452,8 @@ cudaError_t launch_sparse_attn(const Geometry& g, const void* q, const void* k_p
     a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ((n * g.D * 4 + 255) / 256) * 256);
     a.arrivals = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.part_lse) + ((n * 4 + 255) / 256) * 256);
     if (g.G <= 8) {  // the swap-AB kernel merges its splits itself, counting arrivals from zero
-      cudaError_t e = cudaMemsetAsync(a.arrivals, 0, (size_t)g.num_q * 4, s);
+      cudaError_t e = launch_chained(zero_u32_kernel, dim3((g.num_q + 255) / 256), dim3(256), 0, s, a.arrivals,
+                                     g.num_q);
       if (e != cudaSuccess) return e;
     }
   }

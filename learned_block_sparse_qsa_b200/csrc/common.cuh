@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <utility>
 
 #include "../../include/qsa.h"
 
@@ -44,6 +45,38 @@ inline cudaError_t set_smem_once(const void* kernel, int bytes) {
 template <typename Kernel>
 inline cudaError_t set_smem_once(Kernel* k, int bytes) {
   return set_smem_once(reinterpret_cast<const void*>(k), bytes);
+}
+
+// Programmatic dependent launch.  The chained kernels of a layer step (compress, indexer,
+// selection, attention) are launched with launch_chained(): such a kernel may be scheduled while
+// the previous kernel in the stream is still running, so that its launch and start-up overlap the
+// previous kernel's tail.  Every kernel launched that way calls chain_wait() as its first
+// statement, before it reads or writes any global memory, and then chain_release().
+//   chain_wait():    returns once the previous grid in the stream has completed and its memory
+//                    operations are visible (a no-op for an ordinary launch).  Because every
+//                    chained kernel waits before it can complete, completion is transitive along
+//                    the chain.
+//   chain_release(): lets the next chained grid be scheduled (its CTAs then sit in their own
+//                    chain_wait() until this grid completes).  Called after the wait, so at most
+//                    two grids of a chain are resident at a time, and a waiting grid holds no
+//                    tensor memory (every allocation comes after the wait).
+__device__ __forceinline__ void chain_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void chain_release() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

@@ -19,6 +19,8 @@ __global__ void __launch_bounds__(256) compress_kernel(
     const bf16* __restrict__ idx_k, const int32_t* __restrict__ new_seq,
     const int32_t* __restrict__ new_pos, int n_groups, const int32_t* __restrict__ page_table,
     int batch, int max_pages, int num_pages, bf16* __restrict__ kcomp, int32_t* err) {
+  chain_wait();
+  chain_release();
   constexpr int CH = DI / 8;  // 16-byte chunks per key row
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long grp = tid / CH;
@@ -80,21 +82,9 @@ cudaError_t launch_compress(const Geometry& g, const void* idx_k, const int32_t*
   const int grid = (int)((threads + 255) / 256);
   auto* ik = static_cast<const bf16*>(idx_k);
   auto* kc = static_cast<bf16*>(kcomp);
-  switch (g.Di) {
-    case 32:
-      compress_kernel<32><<<grid, 256, 0, s>>>(ik, new_seq, new_pos, n_groups, g.page_table,
-                                               g.batch, g.max_pages, g.num_pages, kc, g.err);
-      break;
-    case 64:
-      compress_kernel<64><<<grid, 256, 0, s>>>(ik, new_seq, new_pos, n_groups, g.page_table,
-                                               g.batch, g.max_pages, g.num_pages, kc, g.err);
-      break;
-    default:
-      compress_kernel<128><<<grid, 256, 0, s>>>(ik, new_seq, new_pos, n_groups, g.page_table,
-                                                g.batch, g.max_pages, g.num_pages, kc, g.err);
-      break;
-  }
-  return cudaGetLastError();
+  auto* kernel = g.Di == 32 ? compress_kernel<32> : g.Di == 64 ? compress_kernel<64> : compress_kernel<128>;
+  return launch_chained(kernel, dim3(grid), dim3(256), 0, s, ik, new_seq, new_pos, n_groups, g.page_table, g.batch,
+                        g.max_pages, g.num_pages, kc, g.err);
 }
 
 }  // namespace qsa

@@ -61,6 +61,8 @@ struct StreamSmem {
 template <int DI>
 __global__ void __launch_bounds__(ST_THREADS, 2)
     score_stream_kernel(ScoreArgs a, u64* __restrict__ cand, int cap, const int32_t* redo) {
+  chain_wait();
+  chain_release();
   using S = StreamSmem<DI>;
   constexpr int CH = DI / 8;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -675,8 +677,8 @@ cudaError_t run_stream(const ScoreArgs& a, const Geometry& g, void* ws, cudaStre
   cudaError_t e = set_smem_once(score_stream_kernel<DI>, smem);
   if (e != cudaSuccess) return e;
   const int tiles = (g.num_q + ST_ROWS - 1) / ST_ROWS;
-  score_stream_kernel<DI><<<tiles, ST_THREADS, smem, s>>>(a, static_cast<u64*>(ws), stream_cap(g.topk), redo);
-  return cudaGetLastError();
+  return launch_chained(score_stream_kernel<DI>, dim3(tiles), dim3(ST_THREADS), smem, s, a, static_cast<u64*>(ws),
+                        stream_cap(g.topk), redo);
 }
 
 MatWs carve_mat(const Geometry& g, void* ws) {

@@ -473,6 +473,8 @@ __global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
     dec_score_kernel(ScoreArgs a, const __grid_constant__ CUtensorMap tmK, DecWs ws, int W, int chunk,
                      int nl) {
   extern __shared__ uint8_t smem_raw[];
+  chain_wait();
+  chain_release();
   dec_score_body<DS_WARPS>(a, &tmK, ws, W, chunk, nl, blockIdx.x, smem_raw, NewBlockWait{});
 }
 
@@ -856,6 +858,8 @@ __device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& 
 
 __global__ void __launch_bounds__(DM_THREADS) dec_merge_kernel(ScoreArgs a, DecWs ws, int nl, int lk) {
   extern __shared__ __align__(128) uint8_t smem[];
+  chain_wait();
+  chain_release();
   dec_merge_body(a, ws, nl, lk, blockIdx.x, smem);
 }
 
@@ -1162,11 +1166,10 @@ cudaError_t launch_score_dec(const ScoreArgs& a, const Geometry& g, void* ws, in
   e = set_smem_once(dec_merge_kernel, MergeSmem::TOTAL);
   if (e != cudaSuccess) return e;
   const int warps = p.T * p.W;
-  dec_score_kernel<<<warps / DS_WARPS, DS_THREADS, DecSmem::TOTAL, s>>>(a, tmK, w, p.W, p.chunk, p.nl);
-  e = cudaGetLastError();
+  e = launch_chained(dec_score_kernel, dim3(warps / DS_WARPS), dim3(DS_THREADS), DecSmem::TOTAL, s, a, tmK, w, p.W,
+                     p.chunk, p.nl);
   if (e != cudaSuccess) return e;
-  dec_merge_kernel<<<g.num_q, DM_THREADS, MergeSmem::TOTAL, s>>>(a, w, p.nl, p.lk);
-  return cudaGetLastError();
+  return launch_chained(dec_merge_kernel, dim3(g.num_q), dim3(DM_THREADS), MergeSmem::TOTAL, s, a, w, p.nl, p.lk);
 }
 
 // ------------------------------------------------------------------ fused decode step (host)

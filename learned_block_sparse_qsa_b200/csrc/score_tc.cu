@@ -299,6 +299,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     score_tc_kernel(ScoreArgs a, const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB, u64* __restrict__ cand,
                     int32_t* __restrict__ redo, TcPlan p) {
+  chain_wait();  // before any global access and before the tensor-memory allocation
+  chain_release();
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sA = smem;
   uint8_t* sB = smem + TC_A_BYTES;
@@ -756,6 +758,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
 // Exclusive prefix of the row tiles' tile counts (one warp), the total last.
 __global__ void tc_scan_kernel(const int32_t* __restrict__ tiles, int R, int32_t* __restrict__ prefix) {
+  chain_wait();
+  chain_release();
   const int lane = threadIdx.x & 31;
   int carry = 0;
   for (int base = 0; base < R; base += 32) {
@@ -786,6 +790,8 @@ static_assert(TS_REGION % 16 == 0 && TS_SMEM <= 232448, "select shared memory");
 
 __global__ void __launch_bounds__(TS_WARPS * 32) tc_select_kernel(ScoreArgs a, TcPlan p,
                                                                  int32_t* __restrict__ redo) {
+  chain_wait();
+  chain_release();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bar[TS_WARPS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -974,8 +980,7 @@ cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int
   TcPlan p{};
   if (!stream) {
     p.mode = 0;
-    score_tc_kernel<<<R, TC_THREADS, TC_SMEM, s>>>(a, tmA, tmB, cand, redo, p);
-    return cudaGetLastError();
+    return launch_chained(score_tc_kernel, dim3(R), dim3(TC_THREADS), TC_SMEM, s, a, tmA, tmB, cand, redo, p);
   }
   const TcStreamWs w = stream_ws_layout(g);
   p.runs = reinterpret_cast<u64*>(wb + w.runs);
@@ -984,16 +989,19 @@ cudaError_t launch_score_tc(const ScoreArgs& a, const Geometry& g, void* ws, int
   p.tiles = reinterpret_cast<int32_t*>(wb + w.tiles);
   p.prefix = reinterpret_cast<int32_t*>(wb + w.prefix);
   p.mode = 1;
-  score_tc_kernel<<<R, TC_THREADS, TC_SMEM, s>>>(a, tmA, tmB, cand, redo, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  tc_scan_kernel<<<1, 32, 0, s>>>(p.tiles, R, p.prefix);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_chained(score_tc_kernel, dim3(R), dim3(TC_THREADS), TC_SMEM, s, a, tmA, tmB, cand, redo, p)) !=
+      cudaSuccess)
+    return e;
+  if ((e = launch_chained(tc_scan_kernel, dim3(1), dim3(32), 0, s, (const int32_t*)p.tiles, R, p.prefix)) !=
+      cudaSuccess)
+    return e;
   p.mode = 2;
-  score_tc_kernel<<<TC_STREAM_CTAS, TC_THREADS, TC_SMEM, s>>>(a, tmA, tmB, cand, redo, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_chained(score_tc_kernel, dim3(TC_STREAM_CTAS), dim3(TC_THREADS), TC_SMEM, s, a, tmA, tmB, cand,
+                          redo, p)) != cudaSuccess)
+    return e;
   if ((e = set_smem_once(tc_select_kernel, TS_SMEM)) != cudaSuccess) return e;
-  tc_select_kernel<<<(g.num_q + TS_WARPS - 1) / TS_WARPS, TS_WARPS * 32, TS_SMEM, s>>>(a, p, redo);
-  return cudaGetLastError();
+  return launch_chained(tc_select_kernel, dim3((g.num_q + TS_WARPS - 1) / TS_WARPS), dim3(TS_WARPS * 32), TS_SMEM, s,
+                        a, p, redo);
 }
 
 }  // namespace qsa
