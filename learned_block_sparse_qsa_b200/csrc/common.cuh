@@ -59,7 +59,8 @@ inline cudaError_t set_smem_once(Kernel* k, int bytes) {
 //   chain_release(): lets the next chained grid be scheduled (its CTAs then sit in their own
 //                    chain_wait() until this grid completes).  Called after the wait, so at most
 //                    two grids of a chain are resident at a time, and a waiting grid holds no
-//                    tensor memory (every allocation comes after the wait).
+//                    tensor memory (every allocation comes after the wait).  A kernel that does
+//                    not call it releases the next grid when it exits.
 __device__ __forceinline__ void chain_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void chain_release() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 

@@ -474,7 +474,9 @@ __global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
                      int nl) {
   extern __shared__ uint8_t smem_raw[];
   chain_wait();
-  chain_release();
+  // No early release: the merge's 16 CTAs, scheduled early, would take the first SMs that free
+  // up, two to an SM; launched at this grid's exit they spread out (C5 graph 97.6 against
+  // 99.6 us with the release).
   dec_score_body<DS_WARPS>(a, &tmK, ws, W, chunk, nl, blockIdx.x, smem_raw, NewBlockWait{});
 }
 
