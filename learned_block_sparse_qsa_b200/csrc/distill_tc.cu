@@ -22,7 +22,7 @@
 //                      lane ends with 2 block sums), added into the block masses of the token in
 //                      global memory (one 8-byte reduction per KV head and block pair).
 //   scores             the indexer scores of every candidate (the materialised scoring kernel).
-//   distill_finish     one warp per row: M = sum m, A = sum m ln m, B = sum m s and the
+//   distill_finish     one CTA per row: M = sum m, A = sum m ln m, B = sum m s and the
 //                      log-sum-exp of s over the candidates; KL = A/M - ln M - B/M + lse(s); the
 //                      teacher m / M when asked for.
 #include "common.cuh"
@@ -376,47 +376,62 @@ __global__ void __launch_bounds__(DK_THREADS, 1)
   }
 }
 
-// One warp per row: the KL from the block masses and the indexer scores of its candidates.  Two
-// sweeps of the row: the largest score, then the sums (per-element logarithms and exponentials in
-// fp32, each lane's sums in fp64).
-__global__ void __launch_bounds__(256) distill_finish_kernel(DkArgs a, const float* __restrict__ scores,
-                                                            long long lds, float* __restrict__ kl,
-                                                            float* __restrict__ teacher, long long ldt) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * 8 + warp;
-  if (r >= a.num_q) return;
+// One 256-thread CTA per row: the KL from the block masses and the indexer scores of its
+// candidates.  Two sweeps of the row: the largest score, then the sums (per-element logarithms and
+// exponentials in fp32, each thread's sums in fp64, reduced over the CTA).
+constexpr int DF_THREADS = 256;
+
+__device__ __forceinline__ double df_block_sum(double v, double* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();  // red[] may still be read by the previous reduction
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  double t = 0.0;
+#pragma unroll
+  for (int w = 0; w < DF_THREADS / 32; ++w) t += red[w];
+  return t;
+}
+
+__global__ void __launch_bounds__(DF_THREADS) distill_finish_kernel(DkArgs a, const float* __restrict__ scores,
+                                                                   long long lds, float* __restrict__ kl,
+                                                                   float* __restrict__ teacher, long long ldt) {
+  __shared__ double red[DF_THREADS / 32];
+  __shared__ float fred[DF_THREADS / 32];
+  const int r = blockIdx.x, tid = threadIdx.x;
   if (!dk_valid(a, r)) {  // flagged by the first launch
-    if (lane == 0) kl[r] = __int_as_float(0x7fc00000);
+    if (tid == 0) kl[r] = __int_as_float(0x7fc00000);
     return;
   }
   const int nb = a.q_pos[r] >> 2;
   const float* mrow = a.mass + (long long)r * a.ldm;
   const float* srow = scores + (long long)r * lds;
   float smax = -INFINITY;
-  for (int b = lane; b < nb; b += 32) smax = fmaxf(smax, srow[b]);
+  for (int b = tid; b < nb; b += DF_THREADS) smax = fmaxf(smax, srow[b]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+  if ((tid & 31) == 0) fred[tid >> 5] = smax;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < DF_THREADS / 32; ++w) smax = fmaxf(smax, fred[w]);
   double M = 0.0, A = 0.0, B = 0.0, Z = 0.0;
-  for (int b = lane; b < nb; b += 32) {
+  for (int b = tid; b < nb; b += DF_THREADS) {
     const float mb = mrow[b], sb = srow[b];
     M += mb;
     if (mb > 1e-30f) A += (double)(mb * __logf(mb));  // below 1e-30 the term is < 1e-28
     B += (double)(mb * sb);
     Z += (double)__expf(sb - smax);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    M += __shfl_xor_sync(0xffffffffu, M, o);
-    A += __shfl_xor_sync(0xffffffffu, A, o);
-    B += __shfl_xor_sync(0xffffffffu, B, o);
-    Z += __shfl_xor_sync(0xffffffffu, Z, o);
-  }
-  if (lane == 0)
+  M = df_block_sum(M, red);
+  A = df_block_sum(A, red);
+  B = df_block_sum(B, red);
+  Z = df_block_sum(Z, red);
+  if (tid == 0)
     kl[r] = (nb > 0 && M > 0.0) ? (float)(A / M - log(M) - B / M + (double)smax + log(Z)) : 0.f;
   if (teacher && nb > 0) {
     const float inv = M > 0.0 ? (float)(1.0 / M) : 0.f;
     float* trow = teacher + (long long)r * ldt;
-    for (int b = lane; b < nb; b += 32) trow[b] = mrow[b] * inv;
+    for (int b = tid; b < nb; b += DF_THREADS) trow[b] = mrow[b] * inv;
   }
 }
 
@@ -482,7 +497,7 @@ cudaError_t launch_distill_tc(const Geometry& g, const void* q, const void* k_po
   distill_tc_kernel<<<dim3((g.num_q + nt - 1) / nt, g.Hkv), DK_THREADS, DK_SMEM, s>>>(a, tmQ, tmK);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = launch_scores_only(g, idx_q, idx_w, kcomp, scores, ldm, s)) != cudaSuccess) return e;
-  distill_finish_kernel<<<(g.num_q + 7) / 8, 256, 0, s>>>(a, scores, ldm, kl, teacher, ld);
+  distill_finish_kernel<<<g.num_q, DF_THREADS, 0, s>>>(a, scores, ldm, kl, teacher, ld);
   return cudaGetLastError();
 }
 
