@@ -42,18 +42,22 @@ __device__ __forceinline__ uint32_t swzd(int r, int c) {
 }
 
 constexpr int DN_NST = 3;
+// Positions per K/V tile of the small-batch (decode) form: half a page, so that a CTA's ring is
+// 48 KB at head_dim 128 and four CTAs share an SM (a whole page: 96 KB, two CTAs, four warps).
+constexpr int kDecPT = 32;
 
-template <int D, int MR>
+template <int D, int MR, int PT>
 struct DenseCfg {
+  static_assert(PT == 32 || PT == 64, "a tile is a page or half a page");
   static constexpr int WARPS = MR / 16;
   static constexpr int THREADS = WARPS * 32;
-  static constexpr int TILE = 64 * D * 2;  // one tensor, one page of one kv head
+  static constexpr int TILE = PT * D * 2;  // one tensor, PT positions of one kv head
   static constexpr int TOTAL = DN_NST * 2 * TILE + 64;
 };
 
-template <int D, int MR>
-__global__ void __launch_bounds__(DenseCfg<D, MR>::THREADS) dense_attn_kernel(DenseArgs a) {
-  using C = DenseCfg<D, MR>;
+template <int D, int MR, int PT>
+__global__ void __launch_bounds__(DenseCfg<D, MR, PT>::THREADS) dense_attn_kernel(DenseArgs a) {
+  using C = DenseCfg<D, MR, PT>;
   constexpr int CH = D / 8;
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sK = smem_addr(smem);
@@ -111,27 +115,28 @@ __global__ void __launch_bounds__(DenseCfg<D, MR>::THREADS) dense_attn_kernel(De
     }
     if (seg < 0) break;
     const bool acta = oka && seqa == seg, actb = okb && seqb == seg;
-    const int npages = tmax / 64 + 1;
-    const int p_lo = (int)((long long)npages * split / a.splits);
-    const int p_hi = (int)((long long)npages * (split + 1) / a.splits);
+    const int ntot = tmax / PT + 1;  // tiles of PT positions up to the segment's last query
+    const int p_lo = (int)((long long)ntot * split / a.splits);
+    const int p_hi = (int)((long long)ntot * (split + 1) / a.splits);
     const int ntiles = p_hi - p_lo;
     const int32_t* ptab = a.page_table + (long long)seg * a.max_pages;
 
     auto load = [&](int it, int st) {
-      const int lp = p_lo + it;
+      const int p0 = (p_lo + it) * PT;  // first position of the tile
+      const int lp = p0 / 64, off = p0 % 64;
       int page = ptab[lp];
       bool ok = page >= 0 && page < a.num_pages;
       if (!ok && tid == 0) flag_error(a.err, QSA_DEVERR_PAGE);
       if (!ok) page = 0;
-      for (int i = tid; i < 2 * 64 * CH; i += C::THREADS) {
-        const int tsr = i / (64 * CH);
-        const int rem = i % (64 * CH);
+      for (int i = tid; i < 2 * PT * CH; i += C::THREADS) {
+        const int tsr = i / (PT * CH);
+        const int rem = i % (PT * CH);
         const int pr = rem / CH, c = rem % CH;
         const bf16* pool = tsr ? a.v_pool : a.k_pool;
-        const bf16* src = pool + (((long long)page * 64 + pr) * a.Hkv + g) * D + c * 8;
+        const bf16* src = pool + (((long long)page * 64 + off + pr) * a.Hkv + g) * D + c * 8;
         // positions past the segment's last query may be unwritten cache slots: zero them so
         // that masked probabilities (0) never meet a non-finite value
-        cp_async16((tsr ? sV : sK) + st * C::TILE + swzd<D>(pr, c), src, ok && lp * 64 + pr <= tmax);
+        cp_async16((tsr ? sV : sK) + st * C::TILE + swzd<D>(pr, c), src, ok && p0 + pr <= tmax);
       }
     };
 
@@ -157,17 +162,17 @@ __global__ void __launch_bounds__(DenseCfg<D, MR>::THREADS) dense_attn_kernel(De
         cp_async_commit();
       }
       const int st = it % DN_NST;
-      const int pbase = (p_lo + it) * 64;
+      const int pbase = (p_lo + it) * PT;
       if (__any_sync(0xffffffffu, tla >= pbase || tlb >= pbase)) {
-        float sc[8][4];
+        float sc[PT / 8][4];
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+        for (int nt = 0; nt < PT / 8; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
 #pragma unroll
-          for (int np = 0; np < 4; ++np) {
+          for (int np = 0; np < PT / 16; ++np) {
             uint32_t kf[4];
             const int pr = np * 16 + (lane & 7) + ((lane >> 4) << 3);
             ldsm_x4(kf, sK + st * C::TILE + swzd<D>(pr, ks * 2 + ((lane >> 3) & 1)));
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(DenseCfg<D, MR>::THREADS) dense_attn_kernel(De
         }
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < PT / 8; ++nt) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int p = pbase + nt * 8 + 2 * qc + e;
@@ -196,7 +201,7 @@ __global__ void __launch_bounds__(DenseCfg<D, MR>::THREADS) dense_attn_kernel(De
         const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
         float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < PT / 8; ++nt) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             sc[nt][e] = mn0 == -INFINITY ? 0.f : exp2f(sc[nt][e] - mn0);
@@ -217,7 +222,7 @@ __global__ void __launch_bounds__(DenseCfg<D, MR>::THREADS) dense_attn_kernel(De
           o[i][3] *= al1;
         }
 #pragma unroll
-        for (int kc = 0; kc < 4; ++kc) {
+        for (int kc = 0; kc < PT / 16; ++kc) {
           uint32_t pf[4];
           pf[0] = pack_bf16(sc[2 * kc][0], sc[2 * kc][1]);
           pf[1] = pack_bf16(sc[2 * kc][2], sc[2 * kc][3]);
@@ -273,14 +278,14 @@ __global__ void __launch_bounds__(DenseCfg<D, MR>::THREADS) dense_attn_kernel(De
   }
 }
 
-template <int D, int MR>
+template <int D, int MR, int PT>
 cudaError_t run_dense(const DenseArgs& a, int splits, cudaStream_t s) {
-  using C = DenseCfg<D, MR>;
-  cudaError_t e = set_smem_once(dense_attn_kernel<D, MR>, C::TOTAL);
+  using C = DenseCfg<D, MR, PT>;
+  cudaError_t e = set_smem_once(dense_attn_kernel<D, MR, PT>, C::TOTAL);
   if (e != cudaSuccess) return e;
   const int TQ = MR / a.G;
   const int tiles = (a.num_q + TQ - 1) / TQ;
-  dense_attn_kernel<D, MR><<<dim3(tiles, a.Hkv, splits), C::THREADS, C::TOTAL, s>>>(a);
+  dense_attn_kernel<D, MR, PT><<<dim3(tiles, a.Hkv, splits), C::THREADS, C::TOTAL, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -289,15 +294,15 @@ cudaError_t run_dense(const DenseArgs& a, int splits, cudaStream_t s) {
 namespace {
 // CTAs of the kernel instance that one SM holds at once (its shared memory decides), looked up
 // once per process; 1 when the runtime cannot say (no device), with the error cleared.
-template <int D, int MR>
+template <int D, int MR, int PT>
 int dense_resident_ctas() {
   static std::atomic<int> cached{0};
   const int c = cached.load(std::memory_order_relaxed);
   if (c > 0) return c;
-  using C = DenseCfg<D, MR>;
+  using C = DenseCfg<D, MR, PT>;
   int n = 0;
-  if (set_smem_once(dense_attn_kernel<D, MR>, C::TOTAL) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dense_attn_kernel<D, MR>, C::THREADS, C::TOTAL) !=
+  if (set_smem_once(dense_attn_kernel<D, MR, PT>, C::TOTAL) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dense_attn_kernel<D, MR, PT>, C::THREADS, C::TOTAL) !=
           cudaSuccess ||
       n < 1) {
     cudaGetLastError();
@@ -317,10 +322,10 @@ int resolve_dense_splits(const Geometry& g, int requested) {
   const int tq = mr / g.G;
   const int tiles = (g.num_q + tq - 1) / tq;
   const int ctas = tiles * g.Hkv;
-  const int per_sm = g.D == 64 ? (small ? dense_resident_ctas<64, 32>() : dense_resident_ctas<64, 64>())
-                               : (small ? dense_resident_ctas<128, 32>() : dense_resident_ctas<128, 64>());
+  const int per_sm = g.D == 64 ? (small ? dense_resident_ctas<64, 32, kDecPT>() : dense_resident_ctas<64, 64, 64>())
+                               : (small ? dense_resident_ctas<128, 32, kDecPT>() : dense_resident_ctas<128, 64, 64>());
   int s = per_sm * num_sms() / ctas;
-  const int pages = g.max_pos / 64 + 1;
+  const int pages = g.max_pos / (small ? kDecPT : 64) + 1;  // at most one tile per split
   if (s > pages) s = pages;
   if (s < 1) s = 1;
   return s;
@@ -365,9 +370,9 @@ cudaError_t launch_dense_attn(const Geometry& g, const void* q, const void* k_po
   const bool small = g.num_q <= 256;
   cudaError_t e;
   if (g.D == 64)
-    e = small ? run_dense<64, 32>(a, splits, s) : run_dense<64, 64>(a, splits, s);
+    e = small ? run_dense<64, 32, kDecPT>(a, splits, s) : run_dense<64, 64, 64>(a, splits, s);
   else
-    e = small ? run_dense<128, 32>(a, splits, s) : run_dense<128, 64>(a, splits, s);
+    e = small ? run_dense<128, 32, kDecPT>(a, splits, s) : run_dense<128, 64, 64>(a, splits, s);
   if (e != cudaSuccess || splits == 1) return e;
   return launch_combine(g, a.part_o, a.part_lse, splits, out, lse, s);
 }

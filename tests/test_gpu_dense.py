@@ -60,3 +60,36 @@ def test_dense_tc_prefill_matches_oracle(name):
         ref_o, ref_lse = oracle_dense_row(c, False, r)
         check_attention(g[r], gl[r], ref_o, ref_lse)
     assert planted or c.ctx % 64 == 0
+
+
+DECODE_CASES = {
+    # 4 sequences x 4 positions; the context ends inside a 32-position tile and a page
+    "g8_b4x4_ctx2531": Config("dense_dec_g8", "decode", 4, 2531, 4, 32, 4, 128, 4, 128,
+                              shuffle_pages=True, seed=0xDE11),
+    "g4_d64_b2x8_ctx1111": Config("dense_dec_g4", "decode", 2, 1111, 8, 16, 4, 64, 4, 64,
+                                  shuffle_pages=True, seed=0xDE12),
+}
+
+
+@pytest.mark.parametrize("splits", [1, 3, 7, 0])
+@pytest.mark.parametrize("name", list(DECODE_CASES))
+def test_dense_decode_all_rows(name, splits):
+    """The decode form (split-K over half-page tiles, merged by log-sum-exp) on every row and head
+    against the oracle; splits 0 is the automatic count that fills the GPU; NaN in the unwritten
+    slots after the last position must not reach the output."""
+    c = DECODE_CASES[name]
+    run = Run(c, integer=False)
+    plant_nan_after_last_position(run)
+    d = run.di
+    out = torch.empty_like(run.out)
+    lse = torch.empty_like(run.lse)
+    run.runner.clear_error()
+    run.runner.dense(run.b, q=d.q, k_pool=d.k_pool, v_pool=d.v_pool, out=out, lse=lse, decode=True,
+                     splits=splits)
+    torch.cuda.synchronize()
+    assert run.runner.error_bits() == 0
+    g = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    gl = lse.cpu().numpy()
+    for r in range(c.num_q):
+        ref_o, ref_lse = oracle_dense_row(c, False, r)
+        check_attention(g[r], gl[r], ref_o, ref_lse)
