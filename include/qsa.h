@@ -98,6 +98,8 @@ typedef struct qsa_config {
                              else the streaming kernel;
                            2 materialised scores (any shape);
                            3 split lists for few rows (idx_dim 128; 2 when its plan does not fit);
+                             the merge launch selects exactly over every candidate itself for a
+                             row the lists cannot settle;
                            4 the mma.sync streaming kernel alone;
                            5 the tcgen05 kernel in its single-launch form, one CTA per 128-row
                              tile (idx_dim 128; 1 otherwise).
@@ -153,8 +155,9 @@ qsa_status_t qsa_index_score_topk(const qsa_config_t* cfg, const qsa_batch_t* ba
                                   int32_t* sel, int32_t* n_sel, float* sel_scores,
                                   void* workspace, size_t ws_bytes, qsa_stream_t stream);
 
-/* Diagnostic, no counterpart in the article.  Paths 1 (idx_dim 128) and 3 first run a fast kernel
- * that settles most rows and flags the rest, which the exact streaming kernel then recomputes.
+/* Diagnostic, no counterpart in the article.  Paths 1 (idx_dim 128), 3 and 5 first run a fast
+ * kernel that settles most rows and flags the rest, which an exact selection then recomputes (the
+ * exact streaming kernel; on path 3 the merge launch itself).
  * This host-only call returns in *flags the device address, inside `workspace`, of those flags
  * (int32 [num_q]: 1 = the row was recomputed, 0 = the fast kernel's own result) as the last
  * qsa_index_score_topk call with this config, batch shape and workspace left them; read them after

@@ -775,11 +775,9 @@ cudaError_t launch_score_topk(const Geometry& g, int path, const void* idx_q, co
       default: return run_stream<128>(a, g, ws, s);
     }
   }
-  if (path == 3) {
+  if (path == 3) {  // the merge kernel runs the exact selection itself for rows it cannot settle
     int32_t* redo = nullptr;
-    cudaError_t e = launch_score_dec(a, g, ws, &redo, s);
-    if (e != cudaSuccess) return e;
-    return run_stream<128>(a, g, ws, s, redo);
+    return launch_score_dec(a, g, ws, &redo, s);
   }
   MatWs w = carve_mat(g, ws);
   mat_clear_kernel<<<64, 256, 0, s>>>(w, g.num_q);

@@ -858,12 +858,6 @@ __device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& 
   }
 }
 
-__global__ void __launch_bounds__(DM_THREADS) dec_merge_kernel(ScoreArgs a, DecWs ws, int nl, int lk) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  chain_wait();
-  chain_release();
-  dec_merge_body(a, ws, nl, lk, blockIdx.x, smem);
-}
 
 // ------------------------------------------------------------------ exact path for one row
 // The row's every candidate score on CUDA cores (4 heads x 128 dims per block), as 64-bit keys in
@@ -988,6 +982,29 @@ __device__ __forceinline__ void inval_mbar(uint8_t* p) {
   asm volatile("mbarrier.inval.shared::cta.b64 [%0];\n" ::"r"(smem_addr(p)) : "memory");
 }
 
+// The merge's mbarrier, inside the MergeSmem layout.
+constexpr int kMergeBarOff = MergeSmem::KEYS + MergeSmem::BOUNDS + MergeSmem::HIST + MergeSmem::CAND +
+                             MergeSmem::LISTS + 448;
+constexpr int kMergeKernelSmem = MergeSmem::TOTAL > ExactSmem::TOTAL ? MergeSmem::TOTAL : ExactSmem::TOTAL;
+
+// One CTA per query row: the split-list merge, and for a row the lists cannot settle, the exact
+// selection over every candidate in the same CTA (exact_keys: the row's candidate keys,
+// exact_ld per row), so that no further launch has to look at the redo flags.
+__global__ void __launch_bounds__(DM_THREADS) dec_merge_kernel(ScoreArgs a, DecWs ws, int nl, int lk,
+                                                              u64* exact_keys, long long exact_ld) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  chain_wait();
+  chain_release();
+  const int row = blockIdx.x;
+  dec_merge_body(a, ws, nl, lk, row, smem);
+  __syncthreads();
+  const bool redo = *reinterpret_cast<volatile int32_t*>(&ws.redo[row]) != 0;
+  if (!redo) return;  // uniform over the CTA
+  if (threadIdx.x == 0) inval_mbar(smem + kMergeBarOff);  // its bytes are reused below
+  __syncthreads();
+  exact_row_body(a, row, exact_keys + (long long)row * exact_ld, smem);
+}
+
 // Bounded wait (thread 0) for *w >= target; then acquire and make generic-proxy writes visible to
 // the async proxy.  Gives up after the wait limit with QSA_DEVERR_TIMEOUT.
 __device__ __forceinline__ void wait_geq(const int* w, int target, int32_t* err) {
@@ -1088,8 +1105,7 @@ __global__ void __launch_bounds__(FS_THREADS, 1)
     __syncthreads();
     dec_merge_body(a, p.ws, p.nl, p.lk, row, smem);
     __syncthreads();
-    if (tid == 0) inval_mbar(smem + MergeSmem::KEYS + MergeSmem::BOUNDS + MergeSmem::HIST + MergeSmem::CAND +
-                             MergeSmem::LISTS + 448);
+    if (tid == 0) inval_mbar(smem + kMergeBarOff);
     const bool redo = *reinterpret_cast<volatile int32_t*>(&p.ws.redo[row]) != 0;
     __syncthreads();
     if (redo) exact_row_body(a, row, p.exact_keys + (long long)row * p.exact_ld, smem);
@@ -1138,11 +1154,19 @@ size_t score_dec_redo_offset(const Geometry& g) {
   return stream_region(g) + r256((size_t)p.T * 4 * p.nl * p.lk * 8) + r256((size_t)p.T * 4 * pad2(p.nl) * 8);
 }
 
+// The three-call form's workspace: the lists, bounds and redo flags, then every row's candidate
+// keys for the merge kernel's exact path ((max_pos/4 + 1) keys per row).
+long long dec_exact_ld(const Geometry& g) { return (long long)g.max_pos / 4 + 1; }
+
+size_t dec_exact_offset(const Geometry& g, const DecPlan& p) {
+  return stream_region(g) + r256((size_t)p.T * 4 * p.nl * p.lk * 8) + r256((size_t)p.T * 4 * pad2(p.nl) * 8) +
+         r256((size_t)g.num_q * 4);
+}
+
 size_t score_dec_workspace_bytes(const Geometry& g) {
   DecPlan p;
   if (!dec_plan(g, &p)) return 0;
-  return stream_region(g) + r256((size_t)p.T * 4 * p.nl * p.lk * 8) +
-         r256((size_t)p.T * 4 * pad2(p.nl) * 8) + r256((size_t)g.num_q * 4);
+  return dec_exact_offset(g, p) + r256((size_t)g.num_q * dec_exact_ld(g) * 8);
 }
 
 cudaError_t launch_score_dec(const ScoreArgs& a, const Geometry& g, void* ws, int32_t** redo_out,
@@ -1165,13 +1189,15 @@ cudaError_t launch_score_dec(const ScoreArgs& a, const Geometry& g, void* ws, in
   }
   cudaError_t e = set_smem_once(dec_score_kernel, DecSmem::TOTAL);
   if (e != cudaSuccess) return e;
-  e = set_smem_once(dec_merge_kernel, MergeSmem::TOTAL);
+  e = set_smem_once(dec_merge_kernel, kMergeKernelSmem);
   if (e != cudaSuccess) return e;
   const int warps = p.T * p.W;
   e = launch_chained(dec_score_kernel, dim3(warps / DS_WARPS), dim3(DS_THREADS), DecSmem::TOTAL, s, a, tmK, w, p.W,
                      p.chunk, p.nl);
   if (e != cudaSuccess) return e;
-  return launch_chained(dec_merge_kernel, dim3(g.num_q), dim3(DM_THREADS), MergeSmem::TOTAL, s, a, w, p.nl, p.lk);
+  u64* exact_keys = reinterpret_cast<u64*>(static_cast<uint8_t*>(ws) + dec_exact_offset(g, p));
+  return launch_chained(dec_merge_kernel, dim3(g.num_q), dim3(DM_THREADS), kMergeKernelSmem, s, a, w, p.nl, p.lk,
+                        exact_keys, dec_exact_ld(g));
 }
 
 // ------------------------------------------------------------------ fused decode step (host)
