@@ -64,6 +64,25 @@ def DISTILL_CONFIG():
                   needles=64, shuffle_pages=True, seed=0x05A6)
 
 
+# The library's kernels per decode step (three calls): compress, the indexer's score and merge
+# launches (the merge runs the exact selection itself for a row it cannot settle), the split-K
+# arrival-counter reset, and the sparse attention.
+DECODE_LAUNCHES_PER_STEP = 5
+
+
+def prefill_launches_per_step(c) -> int:
+    """The library's kernels per prefill step at idx_dim 128 (automatic score path): compress, the
+    tensor-core indexer -- in its stream-K form a sample launch, a scan, the stream launch and a
+    select launch, else one launch -- then the exact-fallback check, and the sparse attention.
+    The form follows the library's geometry rule: stream-K when spreading the row tiles' key tiles
+    over 148 CTAs saves more than its own cost of about 100 tile times."""
+    R = (c.num_q + 127) // 128                   # 128-row tiles
+    T = ((c.ctx - 1) // 4 + 127) // 128 + 1      # 128-block key tiles up to the largest position
+    waves = (R + 147) // 148
+    stream = R * T // 148 + 100 < waves * T
+    return 1 + (4 if stream else 1) + 1 + 1
+
+
 def positions_of(t: int, topk: int = 512) -> int:
     """Token positions attended by query position t: selected blocks plus the clipped tail."""
     n = min(topk, t // 4)
@@ -827,7 +846,7 @@ def main():
     total_ms = max_over_ranks(total_ms, dist)
     ms_step = total_ms / args.steps
     value = job_throughput(world, c.num_q, args.steps, total_ms)
-    launches_per_step = 4  # compress, score + select, exact-fallback check, sparse attention
+    launches_per_step = prefill_launches_per_step(c)
     stages = {
         "compress": dict(ms=stage_ms["compress"], bound="hbm", unit="GB/s",
                          achieved=work["compress_bytes"] / (stage_ms["compress"] * 1e-3) / 1e9,
@@ -941,7 +960,7 @@ def main():
                        "cpu_baseline": dcpu,
                        "e2e": {"value": d_e2e_us, "unit": "us/step", "h2d_bytes_per_step": dh2d,
                                "d2h_bytes_per_step": dd2h},
-                       "gpu_launches_per_step": 5},
+                       "gpu_launches_per_step": DECODE_LAUNCHES_PER_STEP},
         }
         print(json.dumps(line))
     if dist:
