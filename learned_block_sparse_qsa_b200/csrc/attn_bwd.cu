@@ -15,7 +15,8 @@
 //   S^T = K Q^T and dA^T = V dO^T (m16n8k16, K and V from shared memory by ldmatrix);
 //   P^T and dS^T in registers;  dQ^T += K^T dS^T (m16n8k16, dS^T transposed with movmatrix);
 //   dV = P^T dO and dK = scale dS^T Q (m16n8k8, 8 heads deep), added to fp32 gradient pools with
-//   vector atomics, since every row that selected a block contributes to its keys and values.
+//   16-byte vector atomics (lane pairs swap halves of their fragments first), since every row
+//   that selected a block contributes to its keys and values.
 // Selected blocks stream through a 2-stage cp.async ring, a block's 4 positions of all KV heads
 // being one contiguous 4 KB run of its page (16-byte skewed slots, as in the forward).
 #include "common.cuh"
@@ -81,8 +82,20 @@ __device__ __forceinline__ void mma_bf16_1688(float (&d)[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(b0));
 }
 
-__device__ __forceinline__ void red_add2(float* p, float x, float y) {
-  atomicAdd(reinterpret_cast<float2*>(p), make_float2(x, y));
+// Add a fragment's pair of pairs as one 16-byte reduction: the m16n8 accumulator gives lane
+// (qr, qc) dims 2qc, 2qc+1 of rows qr (c0, c1) and qr + 8 (c2, c3); lanes qc and qc ^ 1 swap
+// halves so that the even lane adds dims 2qc..2qc+3 of row qr and the odd lane dims
+// 2qc-2..2qc+1 of row qr + 8.  base_a / base_b: the rows' addresses at dim 0 of this n-tile
+// (nullptr: that row is not added); 16-byte aligned.
+__device__ __forceinline__ void red_add_quad(float* base_a, float* base_b, const float (&c)[4], float scale, int qc) {
+  const bool odd = qc & 1;
+  const float s0 = odd ? c[0] : c[2], s1 = odd ? c[1] : c[3];  // what the partner needs
+  const float r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+  float* dst = odd ? base_b : base_a;
+  if (!dst) return;
+  const float4 v = odd ? make_float4(r0 * scale, r1 * scale, c[2] * scale, c[3] * scale)
+                       : make_float4(c[0] * scale, c[1] * scale, r0 * scale, r1 * scale);
+  atomicAdd(reinterpret_cast<float4*>(dst + 2 * (qc & ~1)), v);
 }
 
 template <int D, int HKV>
@@ -259,15 +272,8 @@ __global__ void __launch_bounds__(BwCfg<D, HKV>::THREADS, 1) sparse_attn_bwd_ker
       float cv[4] = {0.f, 0.f, 0.f, 0.f}, ck[4] = {0.f, 0.f, 0.f, 0.f};
       mma_bf16_1688(cv, pa0, pa1, gn[nt]);
       mma_bf16_1688(ck, sa0, sa1, qn[nt]);
-      const int d = nt * 8 + 2 * qc;
-      if (ra >= 0) {
-        red_add2(a.dv + ra + d, cv[0], cv[1]);
-        red_add2(a.dk + ra + d, ck[0] * a.scale, ck[1] * a.scale);
-      }
-      if (rb >= 0) {
-        red_add2(a.dv + rb + d, cv[2], cv[3]);
-        red_add2(a.dk + rb + d, ck[2] * a.scale, ck[3] * a.scale);
-      }
+      red_add_quad(ra >= 0 ? a.dv + ra + nt * 8 : nullptr, rb >= 0 ? a.dv + rb + nt * 8 : nullptr, cv, 1.f, qc);
+      red_add_quad(ra >= 0 ? a.dk + ra + nt * 8 : nullptr, rb >= 0 ? a.dk + rb + nt * 8 : nullptr, ck, a.scale, qc);
     }
   }
   cp_async_wait<0>();
