@@ -79,11 +79,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Barrier over `n` threads (a multiple of 32) under id `id` (1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
-}
-
 __device__ __forceinline__ bool dk_valid(const DkArgs& a, int r) {
   const int s = a.q_seq[r], t = a.q_pos[r];
   return s >= 0 && s < a.batch && t >= 0 && t <= a.max_pos && t / 64 < a.max_pages;

@@ -780,110 +780,140 @@ __global__ void tc_scan_kernel(const int32_t* __restrict__ tiles, int R, int32_t
 // left for the row, in CTA order (so that each column half's list is ascending by block, with a
 // zero key after each odd-length run, below every real key), staged by bulk copies; then the
 // need-th largest key, the keys at or above it kept in place, and a merge by block.
-constexpr int TS_WARPS = 6;
+// Two warps (a pair) share one key area sized for the largest possible row: when both rows fit
+// in it (the usual case: a row stages about 1,700 of the area's 4,394 slots) they run side by
+// side, the odd warp's keys after the even warp's; otherwise the even warp runs first and hands
+// the area over at the pair's barrier.  Sharing lets ten warps share an SM instead of six.
+constexpr int TS_WARPS = 10;
 constexpr int TS_KEYS = 2 * TC_CAP + 2 * (TC_STREAM_CTAS + 1);  // both halves, odd runs padded
 constexpr int TS_RUNS = 2 * (TC_STREAM_CTAS + 1);                // runs of one row, at most
 constexpr int TS_TABLE = (TS_RUNS * 8 + 15) / 16 * 16;           // (count, offset) per run
-constexpr int TS_REGION = TC_SEL_HIST * 4 + TS_TABLE + TS_KEYS * 8;
-constexpr int TS_SMEM = TS_WARPS * TS_REGION;
-static_assert(TS_REGION % 16 == 0 && TS_SMEM <= 232448, "select shared memory");
+constexpr int TS_WARP_BYTES = TC_SEL_HIST * 4 + TS_TABLE;        // per warp: histogram, run table
+constexpr int TS_SMEM = TS_WARPS * TS_WARP_BYTES + (TS_WARPS / 2) * TS_KEYS * 8;
+static_assert(TS_WARPS % 2 == 0 && TS_WARPS / 2 <= 15, "warp pairs, one named barrier each");
+static_assert(TS_WARP_BYTES % 16 == 0 && TS_SMEM <= 232448, "select shared memory");
 
 __global__ void __launch_bounds__(TS_WARPS * 32) tc_select_kernel(ScoreArgs a, TcPlan p,
                                                                  int32_t* __restrict__ redo) {
   chain_wait();
   chain_release();
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem[];  // the one dynamic buffer of this file
   __shared__ uint64_t bar[TS_WARPS];
+  __shared__ int pair_need[TS_WARPS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < TS_WARPS) mbar_init(&bar[threadIdx.x], 1);
   mbar_fence_init();
   __syncthreads();
   const int row = blockIdx.x * TS_WARPS + warp;
-  if (row >= a.num_q) return;
-  int seq = -1;
-  const int lim = row_limit(a, row, &seq);
-  if (lim < 0) return;  // the sample launch wrote its empty selection
-  uint8_t* region = smem + warp * TS_REGION;
+  uint8_t* region = smem + warp * TS_WARP_BYTES;
   uint32_t* hist = reinterpret_cast<uint32_t*>(region);
   int* table = reinterpret_cast<int*>(region + TC_SEL_HIST * 4);
-  u64* sk = reinterpret_cast<u64*>(region + TC_SEL_HIST * 4 + TS_TABLE);
-  const int need = min(a.topk, lim);
-  if (need == 0) {
-    tc_write_merged(sk, 0, sk, 0, row, lim, a);
-    return;
-  }
-  const int R = (a.num_q + TC_ROWS - 1) / TC_ROWS;
-  const int rt = row / TC_ROWS, rl = row % TC_ROWS;
-  const int total = p.prefix[R];
-  const int W = (total + TC_STREAM_CTAS - 1) / TC_STREAM_CTAS;
-  const int S = p.prefix[rt], T = p.prefix[rt + 1] - S;
-  if (T <= 0 || W <= 0) {  // no tile of this row was streamed: leave it to the exact kernel
-    if (lane == 0) redo[row] = 1;
-    return;
-  }
-  const int c0 = S / W, c1 = (S + T - 1) / W;
-  const int nr = 2 * (c1 - c0 + 1);  // runs: half-major, then CTA order
-  // every lane reads the counts of its runs at once; the staged slots follow by a warp scan
+  u64* pair_keys = reinterpret_cast<u64*>(smem + TS_WARPS * TS_WARP_BYTES) + (size_t)(warp >> 1) * TS_KEYS;
+
+  // ---- this row's runs and staged size; rows with nothing to stage take no key slots
+  bool work = false;
+  int need = 0, lim = -1, nr = 0, c0 = 0, c1 = 0, rt = 0, rl = 0;
   int n[2] = {0, 0}, st[2] = {0, 0};
-  for (int b0 = 0; b0 < nr; b0 += 32) {
-    const int i = b0 + lane;
-    const int h = i / (c1 - c0 + 1), c = c0 + i % (c1 - c0 + 1);
-    const int k = i < nr ? p.runcnt[((long long)(rt + c) * TC_ROWS + rl) * 2 + h] : 0;
-    const int kr = (min(k, TC_CAP) + 1) & ~1;
-    int incl = kr;
+  if (row < a.num_q) {
+    int seq = -1;
+    lim = row_limit(a, row, &seq);  // < 0: the sample launch wrote its empty selection
+    if (lim >= 0) need = min(a.topk, lim);
+    if (lim >= 0 && need == 0) tc_write_merged(pair_keys, 0, pair_keys, 0, row, lim, a);  // no keys read
+    if (lim >= 0 && need > 0) {
+      const int R = (a.num_q + TC_ROWS - 1) / TC_ROWS;
+      rt = row / TC_ROWS;
+      rl = row % TC_ROWS;
+      const int total = p.prefix[R];
+      const int W = (total + TC_STREAM_CTAS - 1) / TC_STREAM_CTAS;
+      const int S = p.prefix[rt], T = p.prefix[rt + 1] - S;
+      if (T <= 0 || W <= 0) {  // no tile of this row was streamed: leave it to the exact kernel
+        if (lane == 0) redo[row] = 1;
+      } else {
+        c0 = S / W;
+        c1 = (S + T - 1) / W;
+        nr = 2 * (c1 - c0 + 1);  // runs: half-major, then CTA order
+        // every lane reads the counts of its runs at once; the staged slots follow by a warp scan
+        for (int b0 = 0; b0 < nr; b0 += 32) {
+          const int i = b0 + lane;
+          const int h = i / (c1 - c0 + 1), c = c0 + i % (c1 - c0 + 1);
+          const int k = i < nr ? p.runcnt[((long long)(rt + c) * TC_ROWS + rl) * 2 + h] : 0;
+          const int kr = (min(k, TC_CAP) + 1) & ~1;
+          int incl = kr;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += u;
-    }
-    if (i < nr) {
-      // staging offset of this run: the slots of every earlier run (earlier chunks included)
-      const int off = st[0] + st[1] + incl - kr;
-      table[2 * i] = k;  // (count, offset) of run i, for the copies and the pads below
-      table[2 * i + 1] = off;
-    }
+          for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+          }
+          if (i < nr && i < TS_RUNS) {
+            // staging offset of this run: the slots of every earlier run (earlier chunks included)
+            const int off = st[0] + st[1] + incl - kr;
+            table[2 * i] = k;  // (count, offset) of run i, for the copies and the pads below
+            table[2 * i + 1] = off;
+          }
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      const bool mine = i < nr && h == h2;
-      int kk = mine ? k : 0, ss = mine ? kr : 0;
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const bool mine = i < nr && h == h2;
+            int kk = mine ? k : 0, ss = mine ? kr : 0;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        kk += __shfl_xor_sync(0xffffffffu, kk, o);
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            for (int o = 16; o > 0; o >>= 1) {
+              kk += __shfl_xor_sync(0xffffffffu, kk, o);
+              ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            }
+            n[h2] += kk;
+            st[h2] += ss;
+          }
+        }
+        if (n[0] > TC_CAP || n[1] > TC_CAP || n[0] + n[1] < need || nr > TS_RUNS) {
+          if (lane == 0) redo[row] = 1;
+        } else {
+          work = true;
+        }
       }
-      n[h2] += kk;
-      st[h2] += ss;
     }
   }
   __syncwarp();
-  if (n[0] > TC_CAP || n[1] > TC_CAP || n[0] + n[1] < need || nr > TS_RUNS) {
-    if (lane == 0) redo[row] = 1;
-    return;
+
+  // ---- the pair's key area: side by side when both rows fit, else the even warp first
+  const int mine = work ? st[0] + st[1] : 0;  // even: 16-byte multiples of slots
+  if (lane == 0) pair_need[warp] = mine;
+  named_bar_sync(1 + (warp >> 1), 64);
+  const int other = pair_need[warp ^ 1];
+  const bool together = mine + other <= TS_KEYS;
+  const bool even = (warp & 1) == 0;
+  u64* sk = pair_keys + (together && !even ? other : 0);
+  if (!together && !even) named_bar_sync(1 + (warp >> 1), 64);  // the even warp is done with it
+
+  if (work) {
+    // the area's earlier generic accesses (the partner's, in the sequential case) come before
+    // the bulk copies' writes
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    if (lane == 0) mbar_arrive_expect_tx(&bar[warp], (uint32_t)(st[0] + st[1]) * 8u);
+    __syncwarp();
+    for (int i = lane; i < nr; i += 32) {  // one lane per run issues its copy
+      const int h = i / (c1 - c0 + 1), c = c0 + i % (c1 - c0 + 1);
+      const int k = table[2 * i], off = table[2 * i + 1];
+      const int kr = (k + 1) & ~1;
+      const long long base = ((long long)(rt + c) * TC_ROWS + rl) * 2 + h;
+      if (kr) bulk_g2s(smem_addr(sk + off), p.runs + base * TC_CAP, (uint32_t)kr * 8u, &bar[warp]);
+    }
+    if (!mbar_wait(&bar[warp], 0, a.err)) {  // (error flagged) wait once more for the copies to land
+      mbar_wait(&bar[warp], 0, a.err);
+      if (lane == 0) redo[row] = 1;
+    } else {
+      for (int i = lane; i < nr; i += 32) {  // the slot after an odd run holds a stale key: below
+        const int k = table[2 * i];          // every real key now
+        if (k & 1) sk[table[2 * i + 1] + k] = 0ull;
+      }
+      __syncwarp();
+      const u64 kth = tc_kth_largest(sk, st[0] + st[1], need, hist);
+      __syncwarp();
+      const int na = tc_keep_inplace(sk, st[0], kth);
+      const int nb = tc_keep_inplace(sk + st[0], st[1], kth);
+      tc_write_merged(sk, na, sk + st[0], nb, row, lim, a);
+    }
   }
-  if (lane == 0) mbar_arrive_expect_tx(&bar[warp], (uint32_t)(st[0] + st[1]) * 8u);
   __syncwarp();
-  for (int i = lane; i < nr; i += 32) {  // one lane per run issues its copy
-    const int h = i / (c1 - c0 + 1), c = c0 + i % (c1 - c0 + 1);
-    const int k = table[2 * i], off = table[2 * i + 1];
-    const int kr = (k + 1) & ~1;
-    const long long base = ((long long)(rt + c) * TC_ROWS + rl) * 2 + h;
-    if (kr) bulk_g2s(smem_addr(sk + off), p.runs + base * TC_CAP, (uint32_t)kr * 8u, &bar[warp]);
-  }
-  if (!mbar_wait(&bar[warp], 0, a.err)) {  // (error flagged) wait once more for the copies to land
-    mbar_wait(&bar[warp], 0, a.err);
-    if (lane == 0) redo[row] = 1;
-    return;
-  }
-  for (int i = lane; i < nr; i += 32) {  // the slot after an odd run holds a stale key: below
-    const int k = table[2 * i];  // every real key now
-    if (k & 1) sk[table[2 * i + 1] + k] = 0ull;
-  }
-  __syncwarp();
-  const u64 kth = tc_kth_largest(sk, st[0] + st[1], need, hist);
-  __syncwarp();
-  const int na = tc_keep_inplace(sk, st[0], kth);
-  const int nb = tc_keep_inplace(sk + st[0], st[1], kth);
-  tc_write_merged(sk, na, sk + st[0], nb, row, lim, a);
+  if (!together && even) named_bar_sync(1 + (warp >> 1), 64);  // hand the area to the odd warp
 }
 
 }  // namespace
