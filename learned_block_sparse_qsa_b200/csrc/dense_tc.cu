@@ -20,7 +20,9 @@
 //               reference maximum in base 2 (raised, with O and the running sum rescaled, only when
 //               a tile's maximum exceeds it by more than 8: lazy rescaling), and write
 //               P = 2^(scale * s - m) as bf16 pairs over the tile's own S columns; at the end
-//               O / l and the log-sum-exp.
+//               O / l and the log-sum-exp.  A tile that every row of the warp sees whole (all but
+//               the last few of a segment) takes a path with no mask code and a three-input
+//               maximum: the softmax's instruction stream, not a pipe, set the pace.
 // Rows of a CTA that belong to different sequences are handled one sequence (segment) at a time.
 // Cache slots after a segment's last position may be unwritten: their V rows are zeroed in the
 // last tile before the MMA reads them, so a masked probability (0) never meets a non-finite value.
@@ -72,6 +74,13 @@ struct DtArgs {
 };
 
 // 2^x on the special-function unit (flush-to-zero, about 2 ulp): plenty for bf16 probabilities.
+// Largest of three (Blackwell's three-input max): half the instructions of a max tree.
+__device__ __forceinline__ float fmax3(float x, float y, float z) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(x), "f"(y), "f"(z));
+  return d;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -283,11 +292,22 @@ __global__ void __launch_bounds__(DT_THREADS, 1)
         // tiles < j)
         waitw(&m->s_full[qt], gj & 1);
         const bool vis = P0 + DT_POS - 1 <= t;  // whole tile visible: no mask
+        const bool allvis = __all_sync(0xffffffffu, vis);  // every row of the warp: no mask code
         // pass 1: the row maximum
         float mx[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
-        if (!dead) {
+        if (!dead && allvis) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < DT_POS / 16; ++c) {
+            float x[16];
+            tmem_ld16(tS + lb + c * 16, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx[e] = fmax3(mx[e], x[e], x[e + 8]);
+          }
+        } else if (!dead) {
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < DT_POS / 16; ++c) {
@@ -330,7 +350,27 @@ __global__ void __launch_bounds__(DT_THREADS, 1)
         float rsv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) rsv[e] = 0.f;
-        if (!dead) {
+        if (!dead && allvis) {
+#pragma unroll
+          for (int c = 0; c < DT_POS / 32; ++c) {
+            float x[16], y[16];
+            tmem_ld16(tS + lb + c * 32, x);
+            tmem_ld16(tS + lb + c * 32 + 16, y);
+            tmem_wait_ld();
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float a0 = e < 8 ? x[2 * e] : y[2 * e - 16];
+              const float a1 = e < 8 ? x[2 * e + 1] : y[2 * e - 15];
+              const float e0 = fast_exp2(fmaf(a0, a.scale_log2, nm));
+              const float e1 = fast_exp2(fmaf(a1, a.scale_log2, nm));
+              rsv[e & 7] += e0 + e1;
+              w[e] = pack_bf16(e0, e1);
+            }
+            tmem_st16u(tS + lb + c * 16, w);
+          }
+          tmem_wait_st();
+        } else if (!dead) {
 #pragma unroll
           for (int c = 0; c < DT_POS / 32; ++c) {
             float x[16], y[16];
