@@ -24,8 +24,9 @@
 // exact top-k whenever no list dropped a key that beats the need-th key of U: a list that dropped
 // keys holds its chunk's 32 largest, so its dropped keys are all below its smallest kept key, and
 // the check is smallest-kept <= tau for every such list.  With random scores a chunk would need
-// more than 16 of the row's top 512 to fail (expected ~1); rows that fail are flagged for the exact
-// streaming kernel, which the caller launches next, so the result never depends on the split.
+// more than 16 of the row's top 512 to fail (expected ~1); a row that fails is flagged, and the
+// same CTA then selects exactly over every candidate of the row (exact_row_body), so the result
+// never depends on the split.
 #include "common.cuh"
 #include "internal.h"
 #include "score_common.cuh"
@@ -115,7 +116,9 @@ struct DecWs {
 
 size_t r256(size_t b) { return (b + 255) / 256 * 256; }
 
-// The exact streaming kernel's candidate buffers come first (it reuses the workspace base).
+// A region the size of the exact streaming kernel's candidate buffers sits at the workspace base
+// (unused by the decode forms: their exact path keeps its keys in a region of its own); the
+// lists, bounds and flags follow it.
 size_t stream_region(const Geometry& g) {
   const int topk = g.topk;
   const int cap = ((4 * topk > topk + 128 ? 4 * topk : topk + 128) + 63) / 64 * 64;
@@ -424,7 +427,7 @@ __device__ __forceinline__ void dec_score_body(const ScoreArgs& a, const CUtenso
     if (aborted) {
       // a page never arrived (reported as QSA_DEVERR_TIMEOUT): wait, bounded, for the copies
       // still in flight into this warp's ring; the maximal bound makes the merge hand the
-      // tile's rows to the exact kernel
+      // tile's rows to the exact path
       for (int j = i; j < min(np, i + DS_NST); ++j)
         mbar_wait(&bar[(base + j) % DS_NST], (uint32_t)((base + j) / DS_NST) & 1u, a.err);
 #pragma unroll
@@ -693,7 +696,7 @@ __device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& 
     bulk_g2s(smem_addr(bnds), ws.bounds + (long long)row * nlp, (uint32_t)(nlp * 8), bar);
   }
   const bool arrived = mbar_wait(bar, 0, a.err);
-  if (!__syncthreads_and(arrived)) {  // reported as a timeout; the exact kernel redoes the row
+  if (!__syncthreads_and(arrived)) {  // reported as a timeout; the exact path redoes the row
     if (tid == 0) {
       ws.redo[row] = 1;
       mbar_wait(bar, 0, a.err);  // and the copies still in flight land first (bounded)
@@ -745,7 +748,7 @@ __device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& 
     hi = y > hi ? y : hi;
     mb = z > mb ? z : mb;
   }
-  if ((int)nk < need) {  // lists dropped too much: the exact kernel redoes the row
+  if ((int)nk < need) {  // lists dropped too much: the exact path redoes the row
     if (tid == 0) ws.redo[row] = 1;
     return;
   }
@@ -819,7 +822,7 @@ __device__ __forceinline__ void dec_merge_body(const ScoreArgs& a, const DecWs& 
                                         wsum, sel3);
     }
   }
-  if (mb > tau) {  // a dropped key could beat tau: the exact kernel redoes the row
+  if (mb > tau) {  // a dropped key could beat tau: the exact path redoes the row
     if (tid == 0) ws.redo[row] = 1;
     return;
   }
