@@ -127,3 +127,19 @@ def test_selftest_rejects_limits_outside_range_before_launch():
     with pytest.raises(q.QsaError) as e:
         q.qsa_selftest_wait_timeout(None, 1_000_000, stream=0)
     assert e.value.status == q.QSA_ERR_INVALID_ARG
+
+
+def test_distill_workspace_contract():
+    """The distillation call's workspace: block masses and indexer scores of every row (fp32,
+    candidates rounded up to 4 per row) in the tensor-core form (head_dim 128, 8 query heads per
+    KV head); none in the other forms.  Without it the tensor-core form refuses to launch."""
+    b = mk_batch(num_q=1024, max_pages=1024, num_pages=1024, max_pos=65535)
+    cfg = q.QsaConfig.make(32, 4, 128, 128)
+    ld = ((65535 // 4 + 1) + 3) // 4 * 4
+    assert q.qsa_workspace_size(cfg, b, q.QSA_OP_DISTILL_KL) == 2 * 1024 * ld * 4
+    for hq, hkv, d in ((32, 4, 64), (32, 2, 128), (8, 8, 128)):  # head_dim 64; 16 and 1 per KV head
+        assert q.qsa_workspace_size(q.QsaConfig.make(hq, hkv, d, 128), b, q.QSA_OP_DISTILL_KL) == 0
+    with pytest.raises(q.QsaError) as e:
+        q.qsa_index_distill_kl(cfg, b, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, stream=0)
+    # QSA_ERR_WORKSPACE, or QSA_ERR_UNSUPPORTED where the driver has no tensor-map encoder (no GPU)
+    assert e.value.status in (q.QSA_ERR_WORKSPACE, q.QSA_ERR_UNSUPPORTED)
