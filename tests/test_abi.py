@@ -143,3 +143,13 @@ def test_distill_workspace_contract():
         q.qsa_index_distill_kl(cfg, b, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, stream=0)
     # QSA_ERR_WORKSPACE, or QSA_ERR_UNSUPPORTED where the driver has no tensor-map encoder (no GPU)
     assert e.value.status in (q.QSA_ERR_WORKSPACE, q.QSA_ERR_UNSUPPORTED)
+
+
+def test_decode_score_workspace_holds_the_exact_path_keys():
+    """The split-list decode indexer (score_path 3, and auto for a few rows) runs the exact
+    selection of a row its lists cannot settle inside the merge launch; the workspace must hold
+    that path's keys: (max_pos/4 + 1) 8-byte keys for every row."""
+    b = mk_batch(num_q=16, batch=4, max_pages=16384, num_pages=65536, max_pos=1048575)
+    for path in (0, 3):
+        cfg = q.QsaConfig.make(32, 4, 128, 128, score_path=path)
+        assert q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK) >= 16 * (1048575 // 4 + 1) * 8
