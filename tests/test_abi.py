@@ -153,3 +153,25 @@ def test_decode_score_workspace_holds_the_exact_path_keys():
     for path in (0, 3):
         cfg = q.QsaConfig.make(32, 4, 128, 128, score_path=path)
         assert q.qsa_workspace_size(cfg, b, q.QSA_OP_INDEX_SCORE_TOPK) >= 16 * (1048575 // 4 + 1) * 8
+
+
+def test_noalloc_automatic_split_count_fits_the_scratch():
+    """qsa_sparse_attn_decode_noalloc with an automatic split count lowers the count until the
+    partials fit its 4 MiB scratch; an explicit count that does not fit is refused.  A shape whose
+    automatic workspace exceeds 4 MiB (64 rows x 64 query heads): the explicit count gets
+    QSA_ERR_WORKSPACE before anything else, the automatic one passes that point and, on a host
+    with no GPU, stops at the launch (QSA_ERR_CUDA).  Host-only: the pointers are not real, so
+    the test never runs where a GPU could launch on them."""
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("host-only: would launch on placeholder pointers")
+    b = mk_batch(num_q=64, max_pages=16384, num_pages=16384, max_pos=1048575)
+    cfg = q.QsaConfig.make(64, 8, 128, 128)
+    assert q.qsa_workspace_size(cfg, b, q.QSA_OP_SPARSE_ATTN_DECODE, 0) > 4 << 20
+    args = (cfg, b, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None)
+    with pytest.raises(q.QsaError) as e:
+        q.qsa_sparse_attn_decode_noalloc(*args, 64, stream=0)
+    assert e.value.status == q.QSA_ERR_WORKSPACE
+    with pytest.raises(q.QsaError) as e:
+        q.qsa_sparse_attn_decode_noalloc(*args, 0, stream=0)
+    assert e.value.status == q.QSA_ERR_CUDA
